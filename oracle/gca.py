@@ -1,0 +1,275 @@
+"""CPU oracle for Geometric Context Attention (GCA).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s cpu_baseline leg and reference arm may import this package.  It
+shares no code with the CUDA library under ``windowed_memory_attention_b200/``
+and never imports it; both sides receive the same seeded inputs from
+``windowed_memory_attention_b200/inputs.py``, which holds no attention
+arithmetic.
+
+Sources (LingBot-Map pages):
+  * paper digest §2.2 (frame-type table): the current frame keeps all M+6
+    tokens; n anchor frames keep all tokens; k pose-reference-window frames keep
+    all tokens; every other earlier frame ("trajectory memory") keeps only its
+    6 summary tokens;
+  * paper digest §2.5 (attention-mask table): the current frame sees anchors
+    (all tokens) + window frames (all tokens) + summary tokens of every history
+    frame; window frames see window + anchors; trajectory-memory frames take
+    part only through their summary tokens;
+  * paper digest §2.4 (token-count formula): cache = M(n+k) + 6T tokens against
+    (M+6)T for causal attention; the worked example M~500, n=3, k=16, T=10000
+    gives about 6.95e4 against about 5.06e6 (~73x);
+  * news article, mask figure caption (d): GCA with n=2 anchors, k=2 window;
+  * code walkthrough §2: a frame that leaves the window drops its M image tokens
+    and keeps its summary tokens; §3.2: anchors ("scale frames") form one block
+    that attends within itself before single-frame streaming.
+
+Readings where the pages leave a step open (each is listed in the design doc):
+  * the k-frame window counts the current frame, so after frame t the full
+    frames are the anchors and t-k+1..t — the only reading under which the
+    cache holds exactly M(n+k)+6T tokens once T > n+k;
+  * attention inside a frame is bidirectional; causality is per frame;
+  * the summary tokens of anchor and window frames are counted once;
+  * in the anchor-block option the n anchors see each other's tokens in full.
+
+Parity pins: tests/test_oracle_pins.py.  The one unpinned quantity is the
+model's learned numbers, which this path does not compute.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from typing import Callable, Iterable, Optional, Sequence
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liboracle.so")
+
+
+# ----------------------------------------------------------------------------
+# closed forms (paper digest §2.4)
+# ----------------------------------------------------------------------------
+def cache_tokens(M: int, S: int, n: int, k: int, T: int) -> int:
+    """Tokens cached by GCA after T frames: full frames hold M image tokens,
+    every frame holds S summary tokens.  Full frames are the first
+    min(T, n+k) frames' worth: n anchors plus the k-frame window."""
+    return M * min(T, n + k) + S * T
+
+
+def causal_tokens(M: int, S: int, T: int) -> int:
+    """Tokens cached by plain causal attention after T frames: (M+S)T."""
+    return (M + S) * T
+
+
+# ----------------------------------------------------------------------------
+# (O2) token-level visibility predicate, paper digest §2.5
+# ----------------------------------------------------------------------------
+def visible(i: int, j: int, tau: int, *, n: int, k: int, S: int,
+            anchor_block: bool = False) -> bool:
+    """May a query token of frame i attend to token slot tau of frame j?
+
+    Slots 0..S-1 are the summary tokens (camera, anchor, 4 registers), slots
+    S..S+M-1 the image tokens.  Frame i itself is part of its window.
+    """
+    if anchor_block and i < n and j < n:
+        return True                       # anchors attend jointly (one block)
+    if j > i:
+        return False                      # no future frames
+    if tau < S:
+        return True                       # summary tokens of every earlier frame
+    return j < n or j >= i - k + 1        # image tokens: anchors and the window
+
+
+# ----------------------------------------------------------------------------
+# (O1) streaming simulator: append frame, evict what left the window
+# ----------------------------------------------------------------------------
+def stream_state(i: int, *, n: int, k: int, anchor_block: bool = False):
+    """Frames holding all tokens, and frames reduced to their summary tokens,
+    in the cache that query frame i reads.
+
+    Replays the stream: frame f enters with all tokens; then every non-anchor
+    frame that is k or more frames behind f drops its image tokens (code
+    walkthrough §2, compressing eviction).  With the anchor block the first n
+    frames enter together, so an anchor query sees all n anchors.
+    """
+    full: set = set()
+    summary: set = set()
+    for f in range(i + 1):
+        full.add(f)
+        for g in sorted(full):
+            if g >= n and g <= f - k:
+                full.discard(g)
+                summary.add(g)
+    if anchor_block and i < n:
+        full |= set(range(n))
+    return sorted(full), sorted(summary)
+
+
+FrameKV = Callable[[int, bool], "tuple[np.ndarray, np.ndarray]"]
+"""frame_kv(j, summary_only) -> (K, V) of frame j for one layer, float32,
+shape [S+M][H][D], or [S][H][D] when summary_only."""
+
+
+def gather_keys(i: int, frame_kv: FrameKV, *, n: int, k: int, S: int,
+                anchor_block: bool = False):
+    """Keys and values that query frame i attends to, [Nk][H][D] float32."""
+    full, summary = stream_state(i, n=n, k=k, anchor_block=anchor_block)
+    ks, vs = [], []
+    for f in full:
+        kf, vf = frame_kv(f, False)
+        ks.append(kf)
+        vs.append(vf)
+    for f in summary:
+        kf, vf = frame_kv(f, True)
+        ks.append(kf[:S])
+        vs.append(vf[:S])
+    return np.concatenate(ks, 0), np.concatenate(vs, 0)
+
+
+# ----------------------------------------------------------------------------
+# attention core: fp64 softmax attention over an explicit key set
+# ----------------------------------------------------------------------------
+def attention_np(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Plain fp64 softmax attention (numpy twin of the C core).
+
+    q [nq][H][D], k and v [nk][H][D]; returns out [nq][H][D] and natural-log
+    lse [nq][H], both float64."""
+    q64 = q.astype(np.float64)
+    k64 = k.astype(np.float64)
+    v64 = v.astype(np.float64)
+    s = scale * np.einsum("rhd,uhd->hru", q64, k64)
+    mx = s.max(axis=2, keepdims=True)
+    p = np.exp(s - mx)
+    den = p.sum(axis=2, keepdims=True)
+    out = np.einsum("hru,uhd->rhd", p, v64) / den.transpose(1, 0, 2)
+    lse = (mx + np.log(den))[:, :, 0].T
+    return out, lse
+
+
+_lib = None
+
+
+def build_core(force: bool = False) -> str:
+    """Compile the C core (gcc, fp64, OpenMP) next to this file."""
+    src = os.path.join(HERE, "gca_oracle.c")
+    if force or not os.path.exists(LIB_PATH) or \
+            os.path.getmtime(LIB_PATH) < os.path.getmtime(src):
+        tmp = LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, src, "-lm"])
+        os.replace(tmp, LIB_PATH)
+    return LIB_PATH
+
+
+def _core():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build_core())
+        lib.gca_oracle_attention.restype = ctypes.c_int
+        lib.gca_oracle_attention.argtypes = [
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_void_p]
+        lib.gca_oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def core_threads() -> int:
+    return int(_core().gca_oracle_num_threads())
+
+
+def attention_c(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """fp64 softmax attention through the C core; same contract as attention_np."""
+    nq, H, D = q.shape
+    nk = k.shape[0]
+    qf = np.ascontiguousarray(q, dtype=np.float32)
+    kh = np.ascontiguousarray(np.asarray(k, dtype=np.float32).transpose(1, 0, 2))
+    vh = np.ascontiguousarray(np.asarray(v, dtype=np.float32).transpose(1, 0, 2))
+    out = np.empty((nq, H, D), dtype=np.float64)
+    lse = np.empty((nq, H), dtype=np.float64)
+    rc = _core().gca_oracle_attention(
+        qf.ctypes.data, nq, kh.ctypes.data, vh.ctypes.data, nk, H, D, float(scale),
+        out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise RuntimeError("oracle core failed")
+    return out, lse
+
+
+def attention(q, k, v, scale, impl: str = "c"):
+    return attention_c(q, k, v, scale) if impl == "c" else attention_np(q, k, v, scale)
+
+
+# ----------------------------------------------------------------------------
+# (O1) one streaming step
+# ----------------------------------------------------------------------------
+def stream_step(q_block: np.ndarray, last_frame: int, frame_kv: FrameKV, *, n: int,
+                k: int, S: int, scale: float, anchor_block: bool = False,
+                rows: Optional[Sequence[int]] = None, impl: str = "c"):
+    """GCA output of the query block that ends at frame ``last_frame``.
+
+    q_block is [F][S+M][H][D] (the F most recent frames' queries).  Returns
+    out [F][R][H][D] and lse [F][R][H] in float64, where R = S+M, or
+    R = len(rows) when ``rows`` picks a subset of each frame's token rows.
+    """
+    F = q_block.shape[0]
+    outs, lses = [], []
+    for b in range(F):
+        i = last_frame - F + 1 + b
+        kk, vv = gather_keys(i, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block)
+        qi = q_block[b] if rows is None else q_block[b][list(rows)]
+        o, l = attention(qi, kk, vv, scale, impl)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+# ----------------------------------------------------------------------------
+# (O2) brute force over the whole sequence with an explicit mask
+# ----------------------------------------------------------------------------
+def visibility_mask(T: int, Lq: int, *, n: int, k: int, S: int,
+                    anchor_block: bool = False) -> np.ndarray:
+    """Boolean [T*Lq][T*Lq] mask of the whole stream from the token rule."""
+    keys = [(j, tau) for j in range(T) for tau in range(Lq)]
+    frame_rows = np.zeros((T, T * Lq), dtype=bool)
+    for i in range(T):
+        for b, (j, tau) in enumerate(keys):
+            frame_rows[i, b] = visible(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block)
+    return np.repeat(frame_rows, Lq, axis=0)
+
+
+def bruteforce(Q: np.ndarray, K: np.ndarray, V: np.ndarray, *, n: int, k: int, S: int,
+               scale: float, anchor_block: bool = False):
+    """Every frame's GCA output at once: Q, K, V [T][S+M][H][D] -> out
+    [T][S+M][H][D], lse [T][S+M][H] (float64)."""
+    T, Lq, H, D = Q.shape
+    q = Q.reshape(T * Lq, H, D).astype(np.float64)
+    kx = K.reshape(T * Lq, H, D).astype(np.float64)
+    vx = V.reshape(T * Lq, H, D).astype(np.float64)
+    mask = visibility_mask(T, Lq, n=n, k=k, S=S, anchor_block=anchor_block)
+    s = scale * np.einsum("rhd,uhd->hru", q, kx)
+    s = np.where(mask[None], s, -np.inf)
+    mx = s.max(axis=2, keepdims=True)
+    p = np.exp(s - mx)
+    den = p.sum(axis=2, keepdims=True)
+    out = np.einsum("hru,uhd->rhd", p, vx) / den.transpose(1, 0, 2)
+    lse = (mx + np.log(den))[:, :, 0].T
+    return out.reshape(T, Lq, H, D), lse.reshape(T, Lq, H)
+
+
+def frame_visibility_matrix(T: int, *, n: int, k: int, S: int, anchor_block: bool = False):
+    """Frame-level picture of the mask: entry [i][j] is 'F' (all tokens of frame
+    j visible to frame i), 'S' (summary tokens only) or '.' (none)."""
+    M_probe = 1
+    rows = []
+    for i in range(T):
+        row = []
+        for j in range(T):
+            summ = visible(i, j, 0, n=n, k=k, S=S, anchor_block=anchor_block)
+            img = visible(i, j, S + M_probe - 1, n=n, k=k, S=S, anchor_block=anchor_block)
+            row.append("F" if img and summ else ("S" if summ else "."))
+        rows.append("".join(row))
+    return rows
