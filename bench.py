@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""GCA hot-path benchmark: frames/sec per layer at T=10000 on the 518x378
+workload (M=999 image + 6 summary tokens, n=3 anchors, k=64 window, H=16,
+D=64, 24 layers, bf16), and the attention kernel's share of the bf16 tensor
+peak.
+
+One step = one new frame through the whole hot path: append its K/V for all
+24 layers (one launch), evict the frame that left the window, then GCA
+attention for each of the 24 layers.  Timed steps are frames 10000-K..9999, so
+the last timed step is at T=10000.  Inputs (seeded synthetic streams) are
+resident in HBM before timing; the end-to-end figure repeats steps with pinned
+host buffers through the same C ABI.
+
+--impl reference times the CPU oracle (oracle/) on the host cores on a bounded
+sample of the same workload (rank 0 only).
+
+Multi-GPU: one independent stream per rank (seeded by rank), no collective on
+the data path (weak scaling); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from windowed_memory_attention_b200 import gca, inputs  # noqa: E402
+
+METRIC = "GCA frames/sec per layer at T=10000 (M=999,n=3,k=64) and % of BF16 TC peak"
+UNIT = "frames/s/layer"
+ATTEND_SRC = os.path.join(ROOT, "windowed_memory_attention_b200", "csrc", "attend_sm100.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU seconds of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"bf16": d["bf16_tflops"], "bf16_sustained": d.get("bf16_tflops_sustained"),
+                "hbm": d["hbm_gbs"], "source": "measured"}
+    except Exception:
+        return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def lk_at(w, T):
+    """Keys a single-frame query sees after T frames: M*min(T, n+k) + S*T."""
+    return w.M * min(T, w.n + w.k) + w.S * T
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if s[4 + i].lower().startswith("active")})
+        loaded = [x for x in sm if mx and x > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+def traffic_record():
+    """dram bytes per attend launch from the committed ncu summary, if it was
+    taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        src = hashlib.sha256(open(ATTEND_SRC, "rb").read()).hexdigest()
+        if rec.get("source_sha256") == src:
+            return rec
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------------------
+# oracle sample (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+class OracleSample:
+    """Layer-0 keys of the step at T=10000, gathered for the CPU oracle."""
+
+    def __init__(self, w):
+        self.w = w
+        self.summ_k, self.summ_v, self.full_k, self.full_v = {}, {}, {}, {}
+
+    def keep_full(self, t, T):
+        return t < self.w.n or t >= T - self.w.k
+
+    def record(self, t, k, v, T):
+        S = self.w.S
+        self.summ_k[t] = k[0, :S].float().cpu().numpy()
+        self.summ_v[t] = v[0, :S].float().cpu().numpy()
+        if self.keep_full(t, T):
+            self.full_k[t] = k[0].float().cpu().numpy()
+            self.full_v[t] = v[0].float().cpu().numpy()
+
+    def run(self, q0, last, rows):
+        """Seconds of one oracle step on `rows`, and its estimate for all rows:
+        (gather of the visible keys, attention of the sampled rows)."""
+        from oracle import gca as ogca
+        w = self.w
+
+        def fkv(j, summary_only):
+            if summary_only:
+                return self.summ_k[j], self.summ_v[j]
+            return self.full_k[j], self.full_v[j]
+        t0 = time.perf_counter()
+        kk, vv = ogca.gather_keys(last, fkv, n=w.n, k=w.k, S=w.S)
+        t1 = time.perf_counter()
+        ogca.attention(q0[rows], kk, vv, w.softmax_scale)
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1
+
+
+def calibrated_rows(sample, q0, last, seconds):
+    g, a = sample.run(q0, last, [0, 1])
+    per_row = a / 2
+    n = int(max(2, min(sample.w.Lq, seconds / max(per_row, 1e-6))))
+    return list(range(n)), per_row
+
+
+# ----------------------------------------------------------------------------
+def run_reference(args):
+    """The CPU oracle as it stands, on the host cores (rank 0 only)."""
+    from oracle import gca as ogca
+    w = inputs.METRIC_518x378
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    T = w.T
+    sample = OracleSample(w)
+    # the synthetic stream is drawn on the GPU when there is one (data only)
+    for t in range(T):
+        k = inputs.draw(w, t, "k", dev)
+        v = inputs.draw(w, t, "v", dev)
+        sample.record(t, k, v, T)
+    q0 = inputs.draw(w, T - 1, "q", dev)[0].float().cpu().numpy()
+    per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    rows, _ = calibrated_rows(sample, q0, T - 1, per_step_s)
+    times = []
+    for i in range(args.warmup + args.steps):
+        g, a = sample.run(q0, T - 1, rows)
+        if i >= args.warmup:
+            times.append(g + a * w.Lq / len(rows))     # estimate of one full layer-step
+    step_s = sum(times) / len(times)
+    value = 1.0 / step_s
+    cores = ogca.core_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * w.L * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "S": w.S, "n": w.n, "k": w.k, "H": w.H,
+                   "D": w.D, "layers": w.L, "T": T},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{len(rows)} query rows x {w.H} heads of layer 0 at T={T} "
+                                   f"(Lk={lk_at(w, T)}) per step: key gather + attention of "
+                                   f"the sampled rows, scaled to all {w.Lq} rows"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    w = inputs.METRIC_518x378.with_(seed0=rank)
+    K, W = args.steps, args.warmup
+    T_end = w.T
+    n_pre = T_end - K - W
+    assert n_pre > w.n + w.k, "too many steps for the stream length"
+    E = max(0, args.e2e_steps)
+    cache = gca.Cache.for_workload(w, max_frames=T_end + E + 2, device=local_rank)
+    stream = torch.cuda.current_stream(dev)
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    sample = OracleSample(w) if want_cpu else None
+
+    # ---- prefill (untimed): frames 0 .. n_pre-1
+    for t in range(n_pre):
+        k = inputs.draw(w, t, "k", dev)
+        v = inputs.draw(w, t, "v", dev)
+        cache.append(k, v)
+        cache.evict()
+        if sample:
+            sample.record(t, k, v, T_end)
+    # ---- inputs of the warm-up and timed steps, resident in HBM
+    frames = []
+    for t in range(n_pre, T_end):
+        k = inputs.draw(w, t, "k", dev)
+        v = inputs.draw(w, t, "v", dev)
+        q = inputs.draw(w, t, "q", dev)
+        frames.append((t, k, v, q))
+        if sample:
+            sample.record(t, k, v, T_end)
+    out = torch.empty((w.L, 1, w.Lq, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+    att_ev = [[(ev(), ev()) for _ in range(w.L)] for _ in range(K)]
+    app_ev = [(ev(), ev()) for _ in range(K)]
+
+    def step(i, timed):
+        t, k, v, q = frames[i]
+        if timed:
+            app_ev[i - W][0].record(stream)
+        cache.append(k, v)
+        if timed:
+            app_ev[i - W][1].record(stream)
+        cache.evict()
+        for l in range(w.L):
+            if timed:
+                att_ev[i - W][l][0].record(stream)
+            cache.attend(l, q[l:l + 1], out[l])
+            if timed:
+                att_ev[i - W][l][1].record(stream)
+
+    for i in range(W):
+        step(i, False)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    launches0 = cache.info().kernel_launches
+    t0, t1 = ev(), ev()
+    t0.record(stream)
+    for i in range(W, W + K):
+        step(i, True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = cache.info().kernel_launches - launches0
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    if cache.status() != 0:
+        raise RuntimeError(f"device status word raised: {cache.status()}")
+
+    att_ms = [a.elapsed_time(b) for s in att_ev for (a, b) in s]
+    app_ms = [a.elapsed_time(b) for (a, b) in app_ev]
+    flops = sum(4.0 * w.Lq * lk_at(w, frames[i][0] + 1) * w.H * w.D
+                for i in range(W, W + K)) * w.L
+    att_total_s = sum(att_ms) / 1e3
+    att_tflops = flops / att_total_s / 1e12
+    app_bytes = 2 * 2 * w.L * w.Lq * w.H * w.D * 2     # K and V, read + write
+    app_gbs = app_bytes / (statistics.mean(app_ms) / 1e3) / 1e9
+
+    # ---- end-to-end: host (pinned) buffers through the same C ABI
+    e2e = None
+    if E > 0:
+        host = []
+        for t in range(T_end, T_end + E + 1):
+            host.append(tuple(inputs.draw(w, t, x, dev).cpu().pin_memory() for x in "kvq"))
+        out_h = torch.empty((w.L, 1, w.Lq, w.H, w.D), dtype=torch.bfloat16).pin_memory()
+
+        def hstep(j):
+            k, v, q = host[j]
+            cache.append(k, v)
+            cache.evict()
+            for l in range(w.L):
+                cache.attend(l, q[l:l + 1], out_h[l])
+
+        hstep(0)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for j in range(1, E + 1):
+            hstep(j)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        fb = w.L * w.Lq * w.H * w.D * 2
+        e2e = {"value": E * w.L * world / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": 3 * fb, "d2h_bytes_per_step": fb}
+
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+
+    if rank != 0:
+        return
+    pk = peaks()
+    tr = traffic_record()
+    value = K * w.L * world / (elapsed_ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "S": w.S, "n": w.n, "k": w.k, "H": w.H,
+                   "D": w.D, "layers": w.L, "T": T_end,
+                   "step": "append all layers + evict + attend per layer",
+                   "parallelism": f"independent stream per GPU x{world}",
+                   "l2": "no flush: per-layer KV is 520 MB and one step reads 12.5 GB, both "
+                         "larger than the 126 MB L2"},
+        "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16"],
+                     "unit": "TFLOP/s", "frac": att_tflops / pk["bf16"],
+                     "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                     "kernel": "gca attend (tcgen05) + merge, per layer launch",
+                     "peak_source": f"{pk['source']} bf16 burst; sustained {pk['bf16_sustained']}",
+                     "algorithmic_flop_per_launch": flops / (K * w.L),
+                     "avg_launch_ms": statistics.mean(att_ms)},
+        "append_roofline": {"bound": "hbm", "achieved": app_gbs, "peak": pk["hbm"],
+                            "unit": "GB/s", "frac": app_gbs / pk["hbm"],
+                            "bytes_per_launch": app_bytes, "avg_launch_ms": statistics.mean(app_ms)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if sample:
+        q0 = frames[-1][3][0].float().cpu().numpy()
+        rows, _ = calibrated_rows(sample, q0, T_end - 1, args.cpu_seconds)
+        g, a = sample.run(q0, T_end - 1, rows)
+        step_s = g + a * w.Lq / len(rows)
+        from oracle import gca as ogca
+        line["cpu_baseline"] = {
+            "value": 1.0 / step_s, "unit": UNIT, "cores": ogca.core_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} query rows x {w.H} heads of layer 0 at T={T_end} "
+                      f"(Lk={lk_at(w, T_end)}): key gather {g:.2f} s + attention {a:.2f} s, "
+                      f"attention scaled to all {w.Lq} rows"}
+    print(json.dumps(line), flush=True)
+    cache.close()
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+/*
+ * gca.h — C ABI of the B200 Geometric Context Attention (GCA) hot path.
+ *
+ * GCA is the cross-frame attention of the Geometric Context Transformer
+ * (LingBot-Map).  Each new frame carries M image-patch tokens and S = 6 summary
+ * tokens (1 camera, 1 anchor, 4 register; paper digest §2.3).  Its queries
+ * attend to three key sets (paper digest §2.2 frame-type table and §2.5
+ * attention-mask table):
+ *   (a) the n anchor frames, all tokens;
+ *   (b) the k most recent frames (the pose-reference window, current frame
+ *       included), all tokens;
+ *   (c) the trajectory memory: only the S summary tokens of every older frame.
+ * The KV cache behind it is paged (news article, inference paragraph; code
+ * walkthrough §3.4) and holds M*min(T, n+k) + S*T tokens after T frames
+ * (paper digest §2.4: M(n+k) + 6T).
+ *
+ * Library-owned state: the page pools (per layer K and V,
+ * [num_pages][H][page_size][D]), one page table shared by all layers, and the
+ * device copy of the walk list.  Caller-owned: every pointer passed to a call.
+ *
+ * Pointers: q, k, v, out and lse may be device pointers or host pointers
+ * (pinned or pageable).  Host inputs are staged through library buffers with
+ * cudaMemcpyAsync on the given stream; host outputs are filled by an async
+ * copy on that stream, so the caller synchronises the stream before reading
+ * them.  Device pointers must stay valid until the stream has consumed them.
+ *
+ * Streams: every GPU step is asynchronous on the stream argument (a
+ * cudaStream_t; NULL = legacy default stream).  Calls on one cache must be
+ * ordered on one stream (or externally synchronised): they share the walk-list
+ * buffer and the scratch space.
+ *
+ * Tensor layouts (row-major, contiguous, dtype of the cache):
+ *   frame tensors  [S+M][H][D]   summary tokens first (camera, anchor,
+ *                                registers), then the M image tokens;
+ *   all-layer form [L][S+M][H][D];
+ *   query block    [F][S+M][H][D] for the F most recent frames;
+ *   lse            [F][S+M][H] float32, natural logarithm.
+ *
+ * Errors: every call returns a gca_status; on error no state changes unless
+ * stated.  GCA_ERR_DEVICE_CHECK reports that a kernel of this cache raised its
+ * device status word (a bounded wait that ran out, or an index check); read it
+ * with gca_device_status.
+ */
+#ifndef GCA_H_
+#define GCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GCA_ALL_LAYERS (-1)
+
+typedef enum {
+    GCA_OK = 0,
+    GCA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad layer index        */
+    GCA_ERR_CAPACITY = 2,      /* page pool or max_frames exhausted              */
+    GCA_ERR_STATE = 3,         /* call out of order (see each call)              */
+    GCA_ERR_UNSUPPORTED = 4,   /* dtype, head_dim or page size not built         */
+    GCA_ERR_CUDA = 5,          /* a CUDA runtime call failed                     */
+    GCA_ERR_DEVICE_CHECK = 6   /* a kernel raised the device status word         */
+} gca_status;
+
+typedef enum { GCA_DTYPE_BF16 = 0, GCA_DTYPE_F32 = 1 } gca_dtype;
+typedef enum { GCA_PAGE_IMAGE = 0, GCA_PAGE_SUMMARY = 1 } gca_page_kind;
+
+typedef struct gca_cache gca_cache_t;  /* opaque, library-owned */
+
+/* Creation parameters.  They mirror the reference constructor's arguments
+ * (resolution -> image_tokens, sliding window, scale frames, tokens per frame,
+ * heads, head_dim, dtype, special-token count; code walkthrough §3.1, §3.4). */
+typedef struct {
+    int32_t num_layers;       /* L >= 1: layers with independent KV streams      */
+    int32_t num_heads;        /* H >= 1                                          */
+    int32_t head_dim;         /* D: 64 (bf16 and f32)                            */
+    int32_t image_tokens;     /* M >= 1: image-patch tokens per frame            */
+    int32_t summary_tokens;   /* S >= 1: summary tokens per frame (6 in GCT)     */
+    int32_t num_anchor;       /* n >= 0: anchor ("scale") frames                 */
+    int32_t window;           /* k >= 1: pose-reference window, current frame in */
+    int32_t max_frames;       /* frames appended before a reset (summary space)  */
+    int32_t page_size;        /* P: 64 or 128 tokens per page                    */
+    int32_t dtype;            /* gca_dtype: BF16 (tcgen05 path), F32 (SIMT path) */
+    int32_t anchor_block;     /* 1: the first n frames attend to each other in
+                                 full (one joint block, code walkthrough §3.2)  */
+    int32_t max_query_frames; /* F_max >= 1: largest query block of gca_attend   */
+    int32_t frame_slack;      /* extra full frames of page space (>= 0)          */
+    float softmax_scale;      /* 0 selects 1/sqrt(D)                             */
+} gca_config_t;
+
+/* One entry of the walk list (the pages gca_attend reads, in order).
+ * Image page: frame = owning frame, first = index of slot 0 among that frame's
+ * image tokens.  Summary page: first = summary-stream index of slot 0 (token s
+ * of frame t has stream index S*t+s), frame = first / S.
+ * n_valid = tokens stored in the page. */
+typedef struct {
+    int32_t page_id;
+    int32_t kind;             /* gca_page_kind */
+    int32_t frame;
+    int32_t first;
+    int32_t n_valid;
+} gca_page_entry_t;
+
+/* Sizes and pool addresses, for tests and tools. */
+typedef struct {
+    int32_t num_pages;        /* pool pages per layer                            */
+    int32_t image_pages_per_frame;
+    int32_t frames;           /* T: frames opened since create / reset           */
+    int32_t full_frames;      /* frames still holding their image pages          */
+    int64_t resident_tokens;  /* M * full_frames + S * T                         */
+    void* k_pool;             /* device: [L][num_pages][H][P][D] of dtype        */
+    void* v_pool;
+    size_t pool_bytes;        /* bytes of one pool (all layers)                  */
+    size_t scratch_bytes;     /* device scratch owned by the cache               */
+    int64_t kernel_launches;  /* kernels this cache has launched since create    */
+} gca_info_t;
+
+/* Create a cache on CUDA device `device`.  Allocates both pools:
+ * num_pages = (n + k + max_query_frames + frame_slack) * ceil(M/P)
+ *           + ceil(S * max_frames / P)  pages per layer.
+ * Errors: INVALID_ARG (non-positive sizes, null out), UNSUPPORTED (head_dim
+ * != 64, page_size not 64/128, unknown dtype), CUDA (allocation). */
+int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out);
+
+/* Free everything the cache owns.  The caller must have synchronised the
+ * streams that used it.  Null is accepted. */
+int gca_cache_destroy(gca_cache_t* cache);
+
+/* Append one frame's K and V (code walkthrough §2: each step adds the new
+ * frame's M+S tokens).  layer == GCA_ALL_LAYERS or 0 opens frame T: the
+ * allocator takes a summary page if the frame's summary tokens start a new one,
+ * then ceil(M/P) image pages, smallest free page id first.  With
+ * GCA_ALL_LAYERS k and v are [L][S+M][H][D] and every layer is written in one
+ * launch; otherwise they are [S+M][H][D] for that layer, and layers 1..L-1
+ * must then append the open frame once each.  *frame_index_out (nullable)
+ * receives the frame index.  Errors: CAPACITY (no pages or max_frames reached;
+ * nothing changes), STATE (layer > 0 with no open frame for it, or layer 0 /
+ * ALL while another layer still misses the open frame). */
+int gca_append_frame(gca_cache_t* cache, int32_t layer, const void* k, const void* v,
+                     int64_t* frame_index_out, void* stream);
+
+/* Compressing eviction (code walkthrough §2; paper-to-code article §2.3):
+ * after frame t, every non-anchor frame f <= t-k that still holds image pages
+ * returns them to the free set.  Its summary tokens stay in the summary stream,
+ * so no bytes move.  Host-only, no stream.  *frames_evicted_out (nullable)
+ * receives the number of frames reduced to summary tokens. */
+int gca_evict_to_summary(gca_cache_t* cache, int32_t* frames_evicted_out);
+
+/* GCA attention for one layer (paper digest §2.5): for the query block of the
+ * F = num_query_frames most recent frames, q [F][S+M][H][D], query frame i
+ * attends to
+ *   every summary token of frames j <= i,
+ *   every image token of frames j <= i with j < n or j >= i-k+1,
+ *   and, with anchor_block, every token of frames j < n when i < n,
+ * with softmax(scale * q.k) over those keys, fp32 accumulation.  out is
+ * [F][S+M][H][D] in the cache dtype; lse (nullable) is [F][S+M][H] float32,
+ * natural log.  Frames needed by the block must not have been evicted: call
+ * gca_evict_to_summary after attending with a block.  Errors: STATE (layer has
+ * not appended frame T-1, F > T, or a needed frame was evicted),
+ * INVALID_ARG (F < 1 or F > max_query_frames), DEVICE_CHECK. */
+int gca_attend(gca_cache_t* cache, int32_t layer, const void* q, int32_t num_query_frames,
+               void* out, float* lse, void* stream);
+
+/* Back to the creation state (windowed mode: state is reset at each window
+ * start; code walkthrough §3.3).  Page tables become identical to a fresh
+ * cache's; pool bytes are left as they are and never read before rewritten. */
+int gca_reset(gca_cache_t* cache);
+
+/* The walk list gca_attend would read for a block of F most recent frames:
+ * image pages of the full frames the block may see (ascending frame, page
+ * order), then every summary page in stream order.  Writes min(n, cap)
+ * entries to out (nullable when cap == 0) and the full count to *n_out. */
+int gca_get_layout(const gca_cache_t* cache, int32_t num_query_frames,
+                   gca_page_entry_t* out, int32_t cap, int32_t* n_out);
+
+/* (page id, slot) of token slot tau of frame `frame` (tau < S: summary).
+ * Errors: INVALID_ARG (frame not appended, tau out of range), STATE (the
+ * frame's image tokens were evicted and tau >= S). */
+int gca_token_slot(const gca_cache_t* cache, int32_t frame, int32_t tau,
+                   int32_t* page_id_out, int32_t* slot_out);
+
+int gca_get_info(const gca_cache_t* cache, gca_info_t* info);
+
+/* Device status word of the cache's kernels (0 = clean) as seen now; it is
+ * complete once the streams that ran them are synchronised.  clear != 0
+ * resets it. */
+int gca_device_status(gca_cache_t* cache, int32_t* status_out, int32_t clear);
+
+/* Static text of a status code. */
+const char* gca_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GCA_H_ */

@@ -1,0 +1,359 @@
+"""GPU parity of the C-ABI library against the CPU oracle.
+
+Every comparison runs the library's kernels through the C ABI on seeded inputs
+and the oracle (oracle/) on the same values.  Tolerances: max |O_gpu - O_oracle|
+<= 1e-4 for the fp32 cache, <= 2e-2 for bf16 inputs with fp32 accumulation;
+page tables and pool bytes bit-exact.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.allocator import PageTableSim
+from windowed_memory_attention_b200 import gca, inputs
+from gca_stream_util import Mirror, attend, max_err, needed_full, oracle_step, pool_view
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+LSE_TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def _sim(w, **kw):
+    return PageTableSim(M=w.M, S=w.S, P=w.page_size, n=w.n, k=w.k,
+                        max_frames=kw.pop("max_frames", w.window_frames or w.T), **kw)
+
+
+def _rows_sample(Lq, extra=0, seed=0):
+    base = {0, 1, 5, 6, 7, 127, 128, 129, 255, 256, Lq // 2, Lq - 2, Lq - 1}
+    rng = np.random.default_rng(seed)
+    base |= set(rng.integers(0, Lq, size=extra).tolist())
+    return sorted(r for r in base if 0 <= r < Lq)
+
+
+# ----------------------------------------------------------------------------
+# tiny workload: every step, full rows, both dtypes
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
+def test_tiny_stream_every_step(w):
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    mirror = Mirror(w, [0])
+    for t in range(w.T):
+        k = inputs.draw(w, t, "k").cuda()
+        v = inputs.draw(w, t, "v").cuda()
+        q = inputs.draw(w, t, "q").cuda()
+        assert cache.append(k, v) == t
+        sim.append()
+        mirror.record(t, k, v, keep_full=True)
+        assert cache.evict() == sim.evict()
+        assert cache.layout() == sim.walk()
+        info = cache.info()
+        assert info.resident_tokens == sim.resident_tokens()
+        out, lse = attend(cache, 0, q)
+        want, wlse = oracle_step(mirror, 0, q.float().cpu().numpy(), t)
+        torch.cuda.synchronize()
+        assert max_err(out, want) <= TOL[w.dtype], t
+        assert max_err(lse, wlse) <= LSE_TOL[w.dtype], t
+    assert cache.status() == 0
+
+
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
+def test_append_writes_pool_bytes_bit_exact(w):
+    cache = gca.Cache.for_workload(w)
+    frames = {}
+    for t in range(w.T):
+        k = inputs.draw(w, t, "k").cuda()
+        v = inputs.draw(w, t, "v").cuda()
+        cache.append(k, v)
+        cache.evict()
+        frames[t] = (k[0].cpu(), v[0].cpu())
+    torch.cuda.synchronize()
+    info = cache.info()
+    P, H, D = w.page_size, w.H, w.D
+    for which, idx in (("k", 0), ("v", 1)):
+        pool = pool_view(cache, which, w.torch_dtype()).view(w.L, info.num_pages, H, P, D).cpu()
+        for t, kv in frames.items():
+            for tau in range(w.Lq):
+                try:
+                    pid, slot = cache.token_slot(t, tau)
+                except gca.GCAError as e:
+                    assert e.name == "GCA_ERR_STATE" and tau >= w.S   # evicted image token
+                    continue
+                got = pool[0, pid, :, slot, :]
+                assert torch.equal(got.view(torch.int16 if w.dtype == "bf16" else torch.int32),
+                                   kv[idx][tau].view(torch.int16 if w.dtype == "bf16" else torch.int32))
+
+
+# ----------------------------------------------------------------------------
+# multi-frame query blocks and the anchor block
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_anchor_block_then_stream(dtype):
+    w = inputs.TINY.with_(dtype=dtype, T=14)
+    cache = gca.Cache.for_workload(w, anchor_block=True, max_query_frames=w.n)
+    sim = _sim(w, anchor_block=True, max_query_frames=w.n)
+    mirror = Mirror(w, [0])
+    qs = []
+    for t in range(w.n):
+        k, v = inputs.draw(w, t, "k").cuda(), inputs.draw(w, t, "v").cuda()
+        cache.append(k, v)
+        sim.append()
+        mirror.record(t, k, v, keep_full=True)
+        qs.append(inputs.draw(w, t, "q").cuda()[0])
+    qb = torch.stack(qs)
+    assert cache.layout(w.n) == sim.walk(w.n)
+    out, lse = attend(cache, 0, qb, F=w.n)
+    want, wlse = oracle_step(mirror, 0, qb.float().cpu().numpy(), w.n - 1, F=w.n, anchor_block=True)
+    torch.cuda.synchronize()
+    assert max_err(out, want) <= TOL[dtype]
+    assert max_err(lse, wlse) <= LSE_TOL[dtype]
+    for t in range(w.n, w.T):
+        k, v, q = (inputs.draw(w, t, x).cuda() for x in "kvq")
+        cache.append(k, v)
+        sim.append()
+        mirror.record(t, k, v, keep_full=True)
+        assert cache.evict() == sim.evict()
+        assert cache.layout() == sim.walk()
+        out, lse = attend(cache, 0, q)
+        want, wlse = oracle_step(mirror, 0, q.float().cpu().numpy(), t, anchor_block=True)
+        torch.cuda.synchronize()
+        assert max_err(out, want) <= TOL[dtype], t
+
+
+@pytest.mark.parametrize("F", [2, 3])
+def test_multi_frame_blocks(F):
+    w = inputs.TINY_BF16.with_(T=20)
+    cache = gca.Cache.for_workload(w, max_query_frames=F)
+    sim = _sim(w, max_query_frames=F)
+    mirror = Mirror(w, [0])
+    t = 0
+    while t + F <= w.T:
+        qs = []
+        for b in range(F):
+            k, v = inputs.draw(w, t + b, "k").cuda(), inputs.draw(w, t + b, "v").cuda()
+            cache.append(k, v)
+            sim.append()
+            mirror.record(t + b, k, v, keep_full=True)
+            qs.append(inputs.draw(w, t + b, "q").cuda()[0])
+        last = t + F - 1
+        assert cache.layout(F) == sim.walk(F)
+        qb = torch.stack(qs)
+        out, lse = attend(cache, 0, qb, F=F)
+        want, wlse = oracle_step(mirror, 0, qb.float().cpu().numpy(), last, F=F)
+        torch.cuda.synchronize()
+        assert max_err(out, want) <= TOL["bf16"], last
+        assert max_err(lse, wlse) <= LSE_TOL["bf16"], last
+        assert cache.evict() == sim.evict()
+        t += F
+
+
+# ----------------------------------------------------------------------------
+# host pointers (the end-to-end path), reset, errors
+# ----------------------------------------------------------------------------
+def test_host_pointer_path_matches_device_path():
+    w = inputs.TINY_BF16
+    a = gca.Cache.for_workload(w)
+    b = gca.Cache.for_workload(w)
+    for t in range(12):
+        k, v, q = (inputs.draw(w, t, x) for x in "kvq")
+        a.append(k.cuda(), v.cuda())
+        b.append(k.pin_memory(), v)                  # pinned and pageable host inputs
+        a.evict()
+        b.evict()
+        out_d, lse_d = attend(a, 0, q.cuda())
+        out_h = torch.empty_like(q).pin_memory()
+        lse_h = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+        b.attend(0, q.pin_memory(), out_h, lse_h)
+        torch.cuda.synchronize()
+        assert torch.equal(out_d.cpu(), out_h)
+        assert torch.equal(lse_d.cpu(), lse_h)
+
+
+def test_reset_gives_fresh_tables_and_outputs():
+    w = inputs.TINY_BF16
+    c = gca.Cache.for_workload(w)
+    fresh = gca.Cache.for_workload(w)
+
+    def run(cache, start, n):
+        outs = []
+        for t in range(start, start + n):
+            k, v, q = (inputs.draw(w, t, x).cuda() for x in "kvq")
+            cache.append(k, v)
+            cache.evict()
+            outs.append((cache.layout(), attend(cache, 0, q)[0]))
+        return outs
+
+    run(c, 0, 20)
+    c.reset()
+    info = c.info()
+    assert info.frames == 0 and info.full_frames == 0 and info.resident_tokens == 0
+    a = run(c, 100, 15)
+    b = run(fresh, 100, 15)
+    torch.cuda.synchronize()
+    for (la, oa), (lb, ob) in zip(a, b):
+        assert la == lb
+        assert torch.equal(oa, ob)
+
+
+def test_state_and_argument_errors():
+    w = inputs.TINY_BF16.with_(L=2)
+    c = gca.Cache.for_workload(w, max_frames=3)
+    q = inputs.draw(w, 0, "q").cuda()
+    out = torch.empty_like(q[0:1].contiguous())
+    with pytest.raises(gca.GCAError) as e:
+        c.attend(0, q[0:1].contiguous(), out)         # nothing appended
+    assert e.value.name == "GCA_ERR_STATE"
+    k, v = inputs.draw(w, 0, "k").cuda(), inputs.draw(w, 0, "v").cuda()
+    with pytest.raises(gca.GCAError) as e:
+        c.append(k[1].contiguous(), v[1].contiguous(), layer=1)   # layer 1 before frame opened
+    assert e.value.name == "GCA_ERR_STATE"
+    c.append(k[0].contiguous(), v[0].contiguous(), layer=0)
+    with pytest.raises(gca.GCAError) as e:
+        c.append(k[0].contiguous(), v[0].contiguous(), layer=0)   # layer 1 still misses frame 0
+    assert e.value.name == "GCA_ERR_STATE"
+    with pytest.raises(gca.GCAError) as e:
+        c.attend(1, q[1:2].contiguous(), out)        # layer 1 has not appended frame 0
+    assert e.value.name == "GCA_ERR_STATE"
+    c.append(k[1].contiguous(), v[1].contiguous(), layer=1)
+    c.attend(1, q[1:2].contiguous(), out)
+    with pytest.raises(gca.GCAError) as e:
+        c.attend(0, q[0:1].contiguous(), out, num_query_frames=2)   # above max_query_frames
+    assert e.value.name == "GCA_ERR_INVALID_ARG"
+    with pytest.raises(gca.GCAError) as e:
+        c.attend(5, q[0:1].contiguous(), out)
+    assert e.value.name == "GCA_ERR_INVALID_ARG"
+    c.append(k, v)
+    c.append(k, v)
+    with pytest.raises(gca.GCAError) as e:
+        c.append(k, v)                               # max_frames = 3
+    assert e.value.name == "GCA_ERR_CAPACITY"
+    assert c.info().frames == 3
+    with pytest.raises(gca.GCAError) as e:
+        gca.Cache(num_layers=1, num_heads=2, image_tokens=16, num_anchor=3, window=4,
+                  max_frames=8, head_dim=128)
+    assert e.value.name == "GCA_ERR_UNSUPPORTED"
+    with pytest.raises(gca.GCAError) as e:
+        gca.Cache(num_layers=0, num_heads=2, image_tokens=16, num_anchor=3, window=4, max_frames=8)
+    assert e.value.name == "GCA_ERR_INVALID_ARG"
+    r = gca.lib().gca_attend(c.handle, 0, None, 1, None, None, None)
+    assert gca.STATUS[r] == "GCA_ERR_INVALID_ARG"
+    assert c.status() == 0
+
+
+def test_page_size_64():
+    w = inputs.TINY_BF16.with_(M=150, page_size=64, T=12)
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    mirror = Mirror(w, [0])
+    for t in range(w.T):
+        k, v, q = (inputs.draw(w, t, x).cuda() for x in "kvq")
+        cache.append(k, v)
+        sim.append()
+        mirror.record(t, k, v, keep_full=True)
+        assert cache.evict() == sim.evict()
+        assert cache.layout() == sim.walk()
+        out, lse = attend(cache, 0, q)
+        want, _ = oracle_step(mirror, 0, q.float().cpu().numpy(), t)
+        torch.cuda.synchronize()
+        assert max_err(out, want) <= TOL["bf16"], t
+
+
+# ----------------------------------------------------------------------------
+# the larger workloads
+# ----------------------------------------------------------------------------
+def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, reset=False):
+    """Stream frames frame0..frame0+T-1 (local indices 0..T-1); at each local
+    step in `checks` compare sampled rows of the listed layers with the oracle."""
+    dev = "cuda"
+    if reset:
+        cache.reset()
+        sim.reset()
+    heads = mirror.heads
+    results = []
+    for t in range(T):
+        g = frame0 + t
+        k = inputs.draw(w, g, "k", dev)
+        v = inputs.draw(w, g, "v", dev)
+        cache.append(k, v)
+        sim.append()
+        keep_full = any(t <= c and (t < w.n or t >= c - w.k + 1) for c in checks)
+        mirror.record(t, k, v, keep_full=keep_full)
+        assert cache.evict() == sim.evict()
+        if t in checks:
+            assert cache.layout() == sim.walk()
+            q = inputs.draw(w, g, "q", dev)
+            for l in layers_to_check:
+                out, lse = attend(cache, l, q[l:l + 1].contiguous())
+                torch.cuda.synchronize()
+                want, wlse = oracle_step(mirror, l, q[l:l + 1].float().cpu().numpy(), t, rows=rows)
+                got, gl = out[0][rows], lse[0][rows]
+                if heads is not None:
+                    got, gl = got[:, heads], gl[:, heads]
+                e = max_err(got, want[0])
+                el = max_err(gl, wlse[0])
+                results.append((t, l, e, el))
+                assert e <= TOL["bf16"], (t, l, e)
+                assert el <= LSE_TOL["bf16"], (t, l, el)
+                assert torch.isfinite(out).all()
+            mirror.drop_full(set(f for f in range(t + 1) if f < w.n) |
+                             set(f for c in checks if c > t for f in range(max(0, c - w.k + 1), t + 1)))
+    assert cache.status() == 0
+    return results
+
+
+def test_worked_example_to_T10000():
+    w = inputs.WORKED_EXAMPLE
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    mirror = Mirror(w, [0])
+    rows = _rows_sample(w.Lq, extra=12)
+    res = _stream(w, cache, sim, mirror, w.T, {99, 999, 9999}, [0], rows)
+    assert cache.info().resident_tokens == 500 * 19 + 6 * 10000
+    print("worked example max errors", res)
+
+
+def test_metric_workload_T10000_all_layers():
+    w = inputs.METRIC_518x378
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    mirror = Mirror(w, [0, 23])
+    rows = _rows_sample(w.Lq, extra=8, seed=3)
+    res = _stream(w, cache, sim, mirror, w.T, {9999}, [0, 23], rows)
+    assert cache.info().resident_tokens == 999 * 67 + 6 * 10000
+    # every layer's output at T=10000 is finite and its lse lies within the
+    # bounds softmax attention allows: ln(#keys) - max|s| <= lse <= ln(#keys) + max|s|
+    q = inputs.draw(w, w.T - 1, "q", "cuda")
+    for l in range(w.L):
+        out, lse = attend(cache, l, q[l:l + 1].contiguous())
+        assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+        assert float(lse.min()) > math.log(126933) - 20 and float(lse.max()) < math.log(126933) + 20
+    print("metric workload max errors", res)
+
+
+def test_windowed_vo_windows():
+    w = inputs.WINDOWED_VO
+    wins = w.windows()
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    rows = _rows_sample(w.Lq, extra=4, seed=5)
+    checks = {0, 1, 2, 3, 66, 67, 68, 127}
+    for idx in (0, 1, len(wins) - 1):
+        start, ln = wins[idx]
+        mirror = Mirror(w, [0])
+        _stream(w, cache, sim, mirror, ln, {c for c in checks if c < ln}, [0], rows,
+                frame0=start, reset=True)
+
+
+def test_dense_causal_limit_T1000():
+    w = inputs.DENSE_CAUSAL
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    heads = [0, 9]
+    mirror = Mirror(w, [0], heads=heads)
+    rows = [0, 5, 6, 500, 1004]
+    res = _stream(w, cache, sim, mirror, w.T, {999}, [0], rows)
+    assert cache.info().resident_tokens == 1005 * 1000
+    print("dense limit errors", res)

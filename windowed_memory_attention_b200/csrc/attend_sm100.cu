@@ -1,0 +1,611 @@
+// GCA attention for sm_100a: tcgen05 tensor cores, TMEM accumulators, TMA.
+//
+// Computes, for every query row r of the block and head h (paper digest §2.5:
+// the current frame attends to anchors and window frames with all tokens and
+// to the summary tokens of every earlier frame),
+//     O[r,h] = softmax_u(scale * q[r,h] . k[u,h]) v[u,h]
+// over the keys of the walk list that row r's frame may see.  Each walk-list
+// page's visible keys are a prefix of its slots (see visible_prefix), so the
+// mask is one integer per (row, page).
+//
+// Work split.  Query rows form QT tiles of 128.  The head-major stream of
+// (head, walk entry) pairs is cut into W contiguous segments; CTA (qt, w)
+// runs query tile qt over segment w.  All QT tiles of a segment read the same
+// K/V pages in the same order at about the same time, so each page comes from
+// HBM once and from L2 for the other tiles.  A segment that covers a whole
+// head writes the final output; heads split between segments leave
+// normalised partials plus their log-sum-exp for the merge kernel.
+//
+// Per CTA (192 threads, one CTA per SM):
+//   warps 0-3  softmax: thread t owns query row t of the tile (TMEM lane t);
+//              loads Q into TMEM, reads S rows from TMEM, online softmax in
+//              the log2 domain with a lazy rescale of O, writes P (bf16) into
+//              TMEM, final normalisation and store;
+//   warp 4     TMA producer: one (page, head) K tile and V tile per stage,
+//              128-byte swizzled boxes of P x 64 bf16, 4 stages;
+//   warp 5     MMA issuer (one thread) and TMEM owner:
+//                S_j  = Q K_j^T   tcgen05.mma kind::f16, A = Q from TMEM,
+//                                 B = K tile (K-major, SW128) from smem;
+//                O   += P_j V_j   A = P from TMEM, B = V tile (MN-major, SW128).
+// TMEM columns: S double buffer (2 x P), P double buffer (2 x P/2 packed
+// bf16x2), O (64), Q (32 packed) — 480 of 512 for P = 128.
+//
+// Every wait on an mbarrier is bounded by a %globaltimer deadline; on expiry
+// the thread raises the CTA abort flag and the device status word, every role
+// leaves its loop, in-flight TMA loads and MMAs are drained (bounded), TMEM is
+// freed and the kernel returns.
+#include <cuda_bf16.h>
+
+#include "gca_internal.h"
+
+namespace gca {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kWarpTMA = 4;
+constexpr int kWarpMMA = 5;
+constexpr int kStages = 4;
+constexpr int kRows = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
+
+template <int PAGE>
+struct Layout {
+    static constexpr int kTileBytes = PAGE * 128;          // PAGE x 64 bf16
+    static constexpr int kStageBytes = 2 * kTileBytes;     // K then V
+    static constexpr int kColS = 0;                        // + buffer * PAGE
+    static constexpr int kColP = 2 * PAGE;                 // + buffer * PAGE/2
+    static constexpr int kColO = 3 * PAGE;
+    static constexpr int kColQ = 3 * PAGE + 64;
+    static_assert(kColQ + 32 <= (int)kTmemCols, "TMEM budget");
+    static constexpr int kNumBars = 2 * kStages + 9;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kNumBars * 8 + 16 + 1024;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+struct Ctl {
+    volatile int* abort;
+    int* status;
+};
+
+// Bounded parity wait.  honour_abort = false is used while draining.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, bool honour_abort = true) {
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 127u) == 0) {
+            if (honour_abort && *c.abort) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                *c.abort = 1;
+                *(volatile int*)c.status = kStatusWaitTimeout;
+                __threadfence_system();
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format:
+// start >> 4 in [0,14), leading byte offset >> 4 in [16,30), stride byte
+// offset >> 4 in [32,46), version 1 at [46,48), swizzle mode 2 at [61,64)).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: D f32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9 = 1, 10-12 = 1), B major at bit 16, N >> 3 at [17,23), M >> 4 at
+// [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d),
+        "r"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+
+#define GCA_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                  "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define GCA_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
+                  "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : GCA_R8(0), GCA_R8(8), GCA_R8(16), GCA_R8(24)
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        GCA_W8(0), GCA_W8(8), GCA_W8(16), GCA_W8(24)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        GCA_W8(0), GCA_W8(8)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <int PAGE>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+              const AttendParams p) {
+    using L = Layout<PAGE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * L::kStageBytes);
+    const uint32_t bar0 = smem_u32(bars);
+    auto kv_full = [&](int s) { return bar0 + 8u * s; };
+    auto kv_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto s_full = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
+    auto s_free = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
+    const uint32_t p_full = bar0 + 8u * (2 * kStages + 4);
+    auto pv_done = [&](int b) { return bar0 + 8u * (2 * kStages + 5 + b); };
+    const uint32_t q_ready = bar0 + 8u * (2 * kStages + 7);
+    const uint32_t drain = bar0 + 8u * (2 * kStages + 8);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Ctl ctl{abort_flag, p.status};
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int qt = blockIdx.x;
+    const int w = blockIdx.y;
+    const long long total = (long long)p.H * p.nwalk;
+    const long long g0 = (long long)w * p.seg;
+    const long long g1 = (g0 + p.seg < total) ? g0 + p.seg : total;
+    const int J = (int)(g1 - g0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(kv_full(s), 1);
+            mbar_init(kv_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full(b), 1);
+            mbar_init(s_free(b), kRows);
+            mbar_init(pv_done(b), 1);
+        }
+        mbar_init(p_full, kRows);
+        mbar_init(q_ready, kRows);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == kWarpTMA && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTMA) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j < J && ok; ++j) {
+                const int st = j % kStages;
+                if (j >= kStages && !wait_bar(kv_empty(st), ((j / kStages) - 1) & 1, ctl)) {
+                    ok = false;
+                    break;
+                }
+                const long long g = g0 + j;
+                const int h = (int)(g / p.nwalk);
+                const int e = (int)(g - (long long)h * p.nwalk);
+                const int page = __ldg(&p.walk[e].x);
+                if (page < 0 || page >= p.num_pages) {
+                    *abort_flag = 1;
+                    *(volatile int*)p.status = kStatusBadPage;
+                    ok = false;
+                    break;
+                }
+                const int y = ((p.layer * p.num_pages + page) * p.H + h) * PAGE;
+                const uint32_t dst = sbase + st * L::kStageBytes;
+                mbar_expect_tx(kv_full(st), 2 * L::kTileBytes);
+                tma_load_2d(dst, &tmK, 0, y, kv_full(st));
+                tma_load_2d(dst + L::kTileBytes, &tmV, 0, y, kv_full(st));
+                ++issued;
+            }
+            if (!ok) {
+                // let every load already issued land before the CTA exits
+                const int from = issued > kStages ? issued - kStages : 0;
+                for (int j = from; j < issued; ++j)
+                    wait_bar(kv_full(j % kStages), (j / kStages) & 1, ctl, false);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kWarpMMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescQK = idesc_bf16(kRows, PAGE, false);
+            constexpr uint32_t kIdescPV = idesc_bf16(kRows, 64, true);
+            bool ok = true;
+            auto issue_pv = [&](int jj) -> bool {
+                if (!wait_bar(p_full, jj & 1, ctl)) return false;
+                fence_after();
+                const int st = jj % kStages;
+                const uint32_t vaddr = sbase + st * L::kStageBytes + L::kTileBytes;
+                const bool first = (jj == 0) || ((g0 + jj) % p.nwalk == 0);
+                const uint32_t pcol = tmem + L::kColP + (jj & 1) * (PAGE / 2);
+#pragma unroll
+                for (int kk = 0; kk < PAGE / 16; ++kk) {
+                    // 16 keys per step: P columns 8kk..8kk+7, V rows 16kk..16kk+15
+                    mma_ts(tmem + L::kColO, pcol + kk * 8,
+                           desc_sw128(vaddr + kk * 2048, L::kTileBytes, 1024), kIdescPV,
+                           (first && kk == 0) ? 0u : 1u);
+                }
+                mma_commit(kv_empty(st));
+                mma_commit(pv_done(jj & 1));
+                return true;
+            };
+            int sidx = 0;
+            for (int j = 0; j < J; ++j) {
+                const bool seg_first = (j == 0) || ((g0 + j) % p.nwalk == 0);
+                if (seg_first) {
+                    if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+                    if (!wait_bar(q_ready, sidx & 1, ctl)) { ok = false; break; }
+                    ++sidx;
+                }
+                const int st = j % kStages;
+                if (!wait_bar(kv_full(st), (j / kStages) & 1, ctl)) { ok = false; break; }
+                if (j >= 2 && !wait_bar(s_free(j & 1), ((j >> 1) - 1) & 1, ctl)) { ok = false; break; }
+                fence_after();
+                const uint32_t kaddr = sbase + st * L::kStageBytes;
+                const uint32_t scol = tmem + L::kColS + (j & 1) * PAGE;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    // 16 head dims per step: Q columns 8kk..8kk+7, K bytes 32kk..32kk+31 of each row
+                    mma_ts(scol, tmem + L::kColQ + kk * 8, desc_sw128(kaddr + kk * 32, 16, 1024),
+                           kIdescQK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full(j & 1));
+                if (!seg_first && !issue_pv(j - 1)) { ok = false; break; }
+            }
+            if (ok) issue_pv(J - 1);
+            // drain: every MMA issued above completes before TMEM is released
+            mma_commit(drain);
+            wait_bar(drain, 0, ctl, false);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int rl = threadIdx.x;                    // row in the tile, TMEM lane
+        const int row = qt * kRows + rl;
+        const bool valid = row < p.R;
+        const int qframe = p.first_query_frame + (valid ? row / p.Lq : 0);
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + L::kColS;
+        const uint32_t t_p = tmem + lane_base + L::kColP;
+        const uint32_t t_o = tmem + lane_base + L::kColO;
+        const uint32_t t_q = tmem + lane_base + L::kColQ;
+        const float sl2 = p.scale_log2;
+        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+
+        auto load_q = [&](int h) {
+            uint32_t r[32];
+            if (valid) {
+                const uint4* src = reinterpret_cast<const uint4*>(qg + ((long long)row * p.H + h) * 64);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 v = __ldg(src + i);
+                    r[4 * i + 0] = v.x;
+                    r[4 * i + 1] = v.y;
+                    r[4 * i + 2] = v.z;
+                    r[4 * i + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = 0u;
+            }
+            tmem_st32(t_q, r);
+            tmem_wait_st();
+            fence_before();
+            mbar_arrive(q_ready);
+        };
+        auto all_ok = [&](bool ok) { return __all_sync(0xffffffffu, ok); };
+
+        float m_run = -INFINITY, l_run = 0.f;
+        load_q((int)(g0 / p.nwalk));
+        for (int j = 0; j < J; ++j) {
+            const long long g = g0 + j;
+            const int h = (int)(g / p.nwalk);
+            const int e = (int)(g - (long long)h * p.nwalk);
+            const bool seg_first = (j == 0) || (e == 0);
+            const bool seg_last = (j == J - 1) || (e == p.nwalk - 1);
+            if (seg_first) {
+                m_run = -INFINITY;
+                l_run = 0.f;
+            }
+            const int4 ent = __ldg(&p.walk[e]);
+            const int nvis = visible_prefix(p.rule, ent, qframe);
+
+            if (!all_ok(wait_bar(s_full(j & 1), (j >> 1) & 1, ctl))) break;
+            fence_after();
+            uint32_t sr[PAGE];
+#pragma unroll
+            for (int c = 0; c < PAGE / 32; ++c) tmem_ld32(t_s + (j & 1) * PAGE + 32 * c, sr + 32 * c);
+            tmem_wait_ld();
+            fence_before();
+            mbar_arrive(s_free(j & 1));
+
+            float s[PAGE];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < PAGE; ++c) {
+                s[c] = (c < nvis) ? __uint_as_float(sr[c]) : -INFINITY;
+                mx = fmaxf(mx, s[c]);
+            }
+            const float mt = mx * sl2;
+            float alpha = 1.f;
+            bool resc = false;
+            if (mt > m_run + kRescaleThreshold) {
+                if (m_run != -INFINITY) {
+                    alpha = ex2(m_run - mt);
+                    resc = true;
+                }
+                m_run = mt;
+            }
+            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+
+            // P buffer (j & 1) was last read by PV_{j-2}
+            if (j >= 2 && !all_ok(wait_bar(pv_done(j & 1), ((j - 2) >> 1) & 1, ctl))) break;
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < PAGE / 32; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, -msub));
+                    const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, -msub));
+                    rs += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
+                }
+                tmem_st16(t_p + (j & 1) * (PAGE / 2) + 16 * c, pk);
+            }
+            l_run = l_run * alpha + rs;
+
+            if (__any_sync(0xffffffffu, resc)) {
+                // O must hold PV_{j-1} before it is rescaled
+                if (!all_ok(wait_bar(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, ctl))) break;
+                fence_after();
+                uint32_t o[64];
+                tmem_ld32(t_o, o);
+                tmem_ld32(t_o + 32, o + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int d = 0; d < 64; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * alpha);
+                tmem_st32(t_o, o);
+                tmem_st32(t_o + 32, o + 32);
+            }
+            tmem_wait_st();
+            fence_before();
+            mbar_arrive(p_full);
+
+            if (seg_last) {
+                if (!all_ok(wait_bar(pv_done(j & 1), (j >> 1) & 1, ctl))) break;
+                fence_after();
+                uint32_t o[64];
+                tmem_ld32(t_o, o);
+                tmem_ld32(t_o + 32, o + 32);
+                tmem_wait_ld();
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                const float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+                const int w_lo = (int)(((long long)h * p.nwalk) / p.seg);
+                const int w_hi = (int)(((long long)(h + 1) * p.nwalk - 1) / p.seg);
+                if (w_lo == w_hi) {
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                              ((long long)row * p.H + h) * 64);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            uint4 v;
+                            v.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+                            v.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+                            v.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+                            v.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+                            dst[i] = v;
+                        }
+                        if (p.lse) p.lse[(long long)row * p.H + h] = lse2 * 0.69314718055994531f;
+                    }
+                } else {
+                    const long long slot = (long long)qt * (p.W + p.H - 1) + w + h;
+                    float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kRows + rl) * 64);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[4 * i + 0]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                             __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+                    p.ws_lse[slot * kRows + rl] = lse2;
+                }
+                if (j < J - 1) load_q(h + 1);
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    fence_before();
+    __syncthreads();
+    if (warp == kWarpMMA) {
+        fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// Combine the partials of heads that were split between workers.
+__global__ void __launch_bounds__(128) merge_kernel(const AttendParams p) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)p.R * p.H) return;
+    const int row = (int)(idx / p.H);
+    const int h = (int)(idx - (long long)row * p.H);
+    const int w_lo = (int)(((long long)h * p.nwalk) / p.seg);
+    const int w_hi = (int)(((long long)(h + 1) * p.nwalk - 1) / p.seg);
+    if (w_lo == w_hi) return;
+    const int qt = row / kRows, rl = row % kRows;
+    const long long base = (long long)qt * (p.W + p.H - 1) + h;
+    float mx = -INFINITY;
+    for (int w = w_lo; w <= w_hi; ++w) mx = fmaxf(mx, p.ws_lse[(base + w) * kRows + rl]);
+    float acc[64];
+#pragma unroll
+    for (int d = 0; d < 64; ++d) acc[d] = 0.f;
+    float den = 0.f;
+    for (int w = w_lo; w <= w_hi; ++w) {
+        const float l2 = p.ws_lse[(base + w) * kRows + rl];
+        if (l2 == -INFINITY) continue;
+        const float wt = exp2f(l2 - mx);
+        den += wt;
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((base + w) * kRows + rl) * 64);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float4 v = src[i];
+            acc[4 * i + 0] += wt * v.x;
+            acc[4 * i + 1] += wt * v.y;
+            acc[4 * i + 2] += wt * v.z;
+            acc[4 * i + 3] += wt * v.w;
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.H + h) * 64);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint4 v;
+        v.x = pack_bf16(acc[8 * i + 0] * inv, acc[8 * i + 1] * inv);
+        v.y = pack_bf16(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv);
+        v.z = pack_bf16(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv);
+        v.w = pack_bf16(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv);
+        dst[i] = v;
+    }
+    if (p.lse) p.lse[(long long)row * p.H + h] = (mx + log2f(den)) * 0.69314718055994531f;
+}
+
+template <int PAGE>
+cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const AttendParams& p,
+                        cudaStream_t s) {
+    const int smem = Layout<PAGE>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel<PAGE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.QT, p.W);
+    attend_kernel<PAGE><<<grid, kThreads, smem, s>>>(tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
+                                const AttendParams& p, cudaStream_t s) {
+    if (p.P == 128) return launch_page<128>(tk, tv, p, s);
+    if (p.P == 64) return launch_page<64>(tk, tv, p, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_merge(const AttendParams& p, cudaStream_t s) {
+    const long long n = (long long)p.R * p.H;
+    merge_kernel<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace gca

@@ -1,0 +1,564 @@
+// C ABI of the GCA hot path: the host page table and the launches.
+//
+// Host state per cache: one page table shared by every layer (the page ids of
+// a frame are the same in all L pools), the frame counter, and for each layer
+// the number of frames it has appended.  Device state: the two pools
+// [L][num_pages][H][P][D], their TMA descriptors, the walk list, the split-KV
+// scratch and the host-mapped status word.
+//
+// Page-table rules (the pages fix only that the cache is paged and sized for
+// scale frames + window + slack; code walkthrough §3.4):
+//   * pages are taken smallest free id first, in token order within a frame:
+//     a new summary page when the frame's summary tokens reach one, then the
+//     frame's ceil(M/P) image pages;
+//   * summary token s of frame t sits at stream index S*t+s, page
+//     (S*t+s)/P of the summary stream, slot (S*t+s)%P;
+//   * eviction after frame t returns the image pages of every non-anchor frame
+//     f <= t-k (code walkthrough §2) — no bytes move;
+//   * the walk list is the image pages of the full frames some query frame of
+//     the block may see (ascending frame, then page), then every summary page.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <set>
+#include <vector>
+
+#include "../../include/gca.h"
+#include "gca_internal.h"
+
+using gca::WalkEntry;
+
+namespace {
+
+constexpr int kRing = 4;       // pinned staging slots for walk-list uploads
+constexpr int kTileRows = 128;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+}  // namespace
+
+struct gca_cache {
+    gca_config_t cfg{};
+    int device = 0;
+    int sms = 148;
+    int P = 128, ipf = 1, num_pages = 0, Lq = 0;
+    size_t elem = 2;
+    float scale = 0.f;
+
+    // page table
+    std::set<int> free_pages;
+    std::map<int, std::vector<int>> image_pages;   // full frames
+    std::vector<int> summary_pages;
+    std::vector<int> summary_opened_by;            // frame that opened each summary page
+    int T = 0;
+    std::vector<int> layer_frames;
+    unsigned long long version = 1;
+
+    // device memory
+    void* kpool = nullptr;
+    void* vpool = nullptr;
+    size_t pool_bytes = 0;
+    CUtensorMap tmK{}, tmV{};
+    WalkEntry* d_walk = nullptr;
+    int walk_cap = 0;
+    WalkEntry* h_stage[kRing] = {};
+    cudaEvent_t stage_ev[kRing] = {};
+    int ring_pos = 0;
+    unsigned long long up_version = 0;
+    int up_F = -1;
+    int up_n = 0;
+    float* ws_o = nullptr;
+    float* ws_lse = nullptr;
+    size_t ws_slots = 0;
+    int* h_status = nullptr;
+    int* d_status = nullptr;
+    // staging for host-memory arguments
+    void* st_k = nullptr;
+    void* st_v = nullptr;
+    void* st_q = nullptr;
+    void* st_out = nullptr;
+    float* st_lse = nullptr;
+    long long launches = 0;
+};
+
+namespace {
+
+void release(gca_cache* c) {
+    if (!c) return;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(c->device);
+    cudaFree(c->kpool);
+    cudaFree(c->vpool);
+    cudaFree(c->d_walk);
+    cudaFree(c->ws_o);
+    cudaFree(c->ws_lse);
+    cudaFree(c->st_k);
+    cudaFree(c->st_v);
+    cudaFree(c->st_q);
+    cudaFree(c->st_out);
+    cudaFree(c->st_lse);
+    for (int i = 0; i < kRing; ++i) {
+        if (c->h_stage[i]) cudaFreeHost(c->h_stage[i]);
+        if (c->stage_ev[i]) cudaEventDestroy(c->stage_ev[i]);
+    }
+    if (c->h_status) cudaFreeHost(c->h_status);
+    cudaSetDevice(prev);
+    delete c;
+}
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        cudaGetDevice(&prev);
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int now = -1;
+        cudaGetDevice(&now);
+        if (prev >= 0 && now != prev) cudaSetDevice(prev);
+    }
+};
+
+bool is_device_ptr(const void* ptr) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+bool encode_pool_map(EncodeTiledFn enc, CUtensorMap* tm, void* pool, const gca_cache* c) {
+    const cuuint64_t rows = (cuuint64_t)c->cfg.num_layers * c->num_pages * c->cfg.num_heads * c->P;
+    cuuint64_t dims[2] = {(cuuint64_t)gca::kHeadDim, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)gca::kHeadDim * 2};
+    cuuint32_t box[2] = {(cuuint32_t)gca::kHeadDim, (cuuint32_t)c->P};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+bool frame_seen(const gca_cache* c, int i, int j) {
+    const int n = c->cfg.num_anchor, k = c->cfg.window;
+    if (c->cfg.anchor_block && i < n && j < n) return true;
+    return j <= i && (j < n || j >= i - k + 1);
+}
+
+// walk list for the block of the F latest frames; false if a needed frame was evicted
+bool build_walk(const gca_cache* c, int F, std::vector<gca_page_entry_t>& out) {
+    out.clear();
+    const int q0 = c->T - F;
+    for (int i = q0; i < c->T; ++i)
+        for (int j = 0; j < c->T; ++j)
+            if (frame_seen(c, i, j) && !c->image_pages.count(j)) return false;
+    for (const auto& kv : c->image_pages) {
+        bool seen = false;
+        for (int i = q0; i < c->T && !seen; ++i) seen = frame_seen(c, i, kv.first);
+        if (!seen) continue;
+        for (size_t s = 0; s < kv.second.size(); ++s) {
+            const int first = (int)s * c->P;
+            out.push_back({kv.second[s], GCA_PAGE_IMAGE, kv.first, first,
+                           std::min(c->P, c->cfg.image_tokens - first)});
+        }
+    }
+    const long long total = (long long)c->cfg.summary_tokens * c->T;
+    for (size_t s = 0; s < c->summary_pages.size(); ++s) {
+        const int first = (int)s * c->P;
+        out.push_back({c->summary_pages[s], GCA_PAGE_SUMMARY, first / c->cfg.summary_tokens, first,
+                       (int)std::min<long long>(c->P, total - first)});
+    }
+    return true;
+}
+
+int check_status(const gca_cache* c) {
+    return (*(volatile int*)c->h_status) ? GCA_ERR_DEVICE_CHECK : GCA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gca_status_string(int s) {
+    switch (s) {
+        case GCA_OK: return "ok";
+        case GCA_ERR_INVALID_ARG: return "invalid argument";
+        case GCA_ERR_CAPACITY: return "capacity exhausted";
+        case GCA_ERR_STATE: return "call out of order";
+        case GCA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case GCA_ERR_CUDA: return "CUDA error";
+        case GCA_ERR_DEVICE_CHECK: return "device status word raised";
+        default: return "unknown status";
+    }
+}
+
+int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
+    if (!cfg || !out) return GCA_ERR_INVALID_ARG;
+    *out = nullptr;
+    const gca_config_t& g = *cfg;
+    if (g.num_layers < 1 || g.num_heads < 1 || g.image_tokens < 1 || g.summary_tokens < 1 ||
+        g.num_anchor < 0 || g.window < 1 || g.max_frames < 1 || g.max_query_frames < 1 ||
+        g.frame_slack < 0 || g.softmax_scale < 0.f)
+        return GCA_ERR_INVALID_ARG;
+    if (g.head_dim != gca::kHeadDim || (g.page_size != 64 && g.page_size != 128) ||
+        (g.dtype != GCA_DTYPE_BF16 && g.dtype != GCA_DTYPE_F32))
+        return GCA_ERR_UNSUPPORTED;
+    if ((g.image_tokens + g.page_size - 1) / g.page_size > gca::kMaxImagePages)
+        return GCA_ERR_UNSUPPORTED;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+        cudaGetLastError();
+        return GCA_ERR_INVALID_ARG;
+    }
+    DeviceGuard guard(device);
+
+    gca_cache* c = new gca_cache();
+    c->cfg = g;
+    c->device = device;
+    cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, device);
+    c->P = g.page_size;
+    c->ipf = ceil_div(g.image_tokens, c->P);
+    const long long image_cap = (long long)(g.num_anchor + g.window + g.max_query_frames + g.frame_slack) * c->ipf;
+    const long long summary_cap = ceil_div((long long)g.summary_tokens * g.max_frames, c->P);
+    if (image_cap + summary_cap > (1LL << 30)) { delete c; return GCA_ERR_CAPACITY; }
+    c->num_pages = (int)(image_cap + summary_cap);
+    c->Lq = g.image_tokens + g.summary_tokens;
+    c->elem = g.dtype == GCA_DTYPE_BF16 ? 2 : 4;
+    c->scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.0f / sqrtf((float)g.head_dim);
+    c->layer_frames.assign(g.num_layers, 0);
+    for (int i = 0; i < c->num_pages; ++i) c->free_pages.insert(i);
+
+    const size_t tile = (size_t)c->P * gca::kHeadDim * c->elem;
+    c->pool_bytes = (size_t)g.num_layers * c->num_pages * g.num_heads * tile;
+    bool ok = cudaMalloc(&c->kpool, c->pool_bytes) == cudaSuccess &&
+              cudaMalloc(&c->vpool, c->pool_bytes) == cudaSuccess;
+    c->walk_cap = c->num_pages;
+    ok = ok && cudaMalloc(&c->d_walk, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess;
+    for (int i = 0; ok && i < kRing; ++i) {
+        ok = cudaHostAlloc((void**)&c->h_stage[i], sizeof(WalkEntry) * c->walk_cap, cudaHostAllocDefault) == cudaSuccess &&
+             cudaEventCreateWithFlags(&c->stage_ev[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    // split-KV scratch: per query tile at most W + H - 1 (worker, head) partials,
+    // with QT * W <= max(SMs, QT)
+    const int qt_max = ceil_div((long long)g.max_query_frames * c->Lq, kTileRows);
+    c->ws_slots = (size_t)std::max(c->sms, qt_max) + (size_t)qt_max * (g.num_heads - 1);
+    if (g.dtype == GCA_DTYPE_BF16) {
+        ok = ok && cudaMalloc(&c->ws_o, c->ws_slots * kTileRows * gca::kHeadDim * sizeof(float)) == cudaSuccess &&
+             cudaMalloc(&c->ws_lse, c->ws_slots * kTileRows * sizeof(float)) == cudaSuccess;
+    }
+    ok = ok && cudaHostAlloc((void**)&c->h_status, sizeof(int), cudaHostAllocMapped) == cudaSuccess;
+    if (ok) {
+        *c->h_status = 0;
+        ok = cudaHostGetDevicePointer((void**)&c->d_status, c->h_status, 0) == cudaSuccess;
+    }
+    const size_t frame_bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
+    ok = ok && cudaMalloc(&c->st_k, frame_bytes * g.num_layers) == cudaSuccess &&
+         cudaMalloc(&c->st_v, frame_bytes * g.num_layers) == cudaSuccess &&
+         cudaMalloc(&c->st_q, frame_bytes * g.max_query_frames) == cudaSuccess &&
+         cudaMalloc(&c->st_out, frame_bytes * g.max_query_frames) == cudaSuccess &&
+         cudaMalloc((void**)&c->st_lse, (size_t)c->Lq * g.num_heads * g.max_query_frames * sizeof(float)) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        release(c);
+        return GCA_ERR_CUDA;
+    }
+    if (g.dtype == GCA_DTYPE_BF16) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            !fn || !encode_pool_map((EncodeTiledFn)fn, &c->tmK, c->kpool, c) ||
+            !encode_pool_map((EncodeTiledFn)fn, &c->tmV, c->vpool, c)) {
+            cudaGetLastError();
+            release(c);
+            return GCA_ERR_CUDA;
+        }
+    }
+    *out = c;
+    return GCA_OK;
+}
+
+int gca_cache_destroy(gca_cache_t* c) {
+    release(c);
+    return GCA_OK;
+}
+
+int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v,
+                     int64_t* frame_index_out, void* stream) {
+    if (!c || !k || !v) return GCA_ERR_INVALID_ARG;
+    const gca_config_t& g = c->cfg;
+    if (layer != GCA_ALL_LAYERS && (layer < 0 || layer >= g.num_layers)) return GCA_ERR_INVALID_ARG;
+    if (int s = check_status(c)) return s;
+    DeviceGuard guard(c->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    int t, l0, nl;
+    if (layer == GCA_ALL_LAYERS || layer == 0) {
+        for (int l = 0; l < g.num_layers; ++l)
+            if (c->layer_frames[l] != c->T) return GCA_ERR_STATE;
+        if (c->T >= g.max_frames) return GCA_ERR_CAPACITY;
+        t = c->T;
+        const int S = g.summary_tokens;
+        int new_sum = 0;
+        for (int s = 0; s < S; ++s) new_sum += ((S * t + s) % c->P) == 0;
+        if ((int)c->free_pages.size() < c->ipf + new_sum) return GCA_ERR_CAPACITY;
+        auto take = [&]() {
+            const int pid = *c->free_pages.begin();
+            c->free_pages.erase(c->free_pages.begin());
+            return pid;
+        };
+        for (int s = 0; s < S; ++s)
+            if (((S * t + s) % c->P) == 0) {
+                c->summary_pages.push_back(take());
+                c->summary_opened_by.push_back(t);
+            }
+        std::vector<int> pages(c->ipf);
+        for (int i = 0; i < c->ipf; ++i) pages[i] = take();
+        c->image_pages[t] = pages;
+        c->T += 1;
+        c->version += 1;
+        l0 = 0;
+        nl = layer == GCA_ALL_LAYERS ? g.num_layers : 1;
+    } else {
+        if (c->T == 0 || c->layer_frames[layer] != c->T - 1) return GCA_ERR_STATE;
+        t = c->T - 1;
+        l0 = layer;
+        nl = 1;
+    }
+
+    gca::AppendParams p{};
+    const size_t bytes = (size_t)nl * c->Lq * g.num_heads * gca::kHeadDim * c->elem;
+    p.k = k;
+    p.v = v;
+    if (!is_device_ptr(k)) {
+        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        p.k = c->st_k;
+    }
+    if (!is_device_ptr(v)) {
+        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        p.v = c->st_v;
+    }
+    p.kpool = c->kpool;
+    p.vpool = c->vpool;
+    p.layer0 = l0;
+    p.nlayers = nl;
+    p.Lq = c->Lq;
+    p.S = g.summary_tokens;
+    p.M = g.image_tokens;
+    p.H = g.num_heads;
+    p.P = c->P;
+    p.num_pages = c->num_pages;
+    p.elem_bytes = (int)c->elem;
+    p.frame = t;
+    const int S = g.summary_tokens;
+    p.sum_seq0 = (S * t) / c->P;
+    p.sum_page[0] = c->summary_pages[p.sum_seq0];
+    p.sum_page[1] = (p.sum_seq0 + 1 < (int)c->summary_pages.size()) ? c->summary_pages[p.sum_seq0 + 1] : -1;
+    p.new_sum_seq = -1;
+    for (int s = 0; s < S; ++s)
+        if (((S * t + s) % c->P) == 0) p.new_sum_seq = (S * t + s) / c->P;
+    const std::vector<int>& img = c->image_pages.at(t);
+    for (int i = 0; i < c->ipf; ++i) p.img_pages[i] = img[i];
+    if (gca::launch_append(p, st) != cudaSuccess) {
+        cudaGetLastError();
+        return GCA_ERR_CUDA;
+    }
+    c->launches += 1;
+    for (int l = l0; l < l0 + nl; ++l) c->layer_frames[l] = t + 1;
+    if (frame_index_out) *frame_index_out = t;
+    return GCA_OK;
+}
+
+int gca_evict_to_summary(gca_cache_t* c, int32_t* frames_evicted_out) {
+    if (!c) return GCA_ERR_INVALID_ARG;
+    const int t = c->T - 1;
+    int count = 0;
+    for (auto it = c->image_pages.begin(); it != c->image_pages.end();) {
+        const int f = it->first;
+        if (f >= c->cfg.num_anchor && f <= t - c->cfg.window) {
+            for (int pid : it->second) c->free_pages.insert(pid);
+            it = c->image_pages.erase(it);
+            ++count;
+        } else {
+            ++it;
+        }
+    }
+    if (count) c->version += 1;
+    if (frames_evicted_out) *frames_evicted_out = count;
+    return GCA_OK;
+}
+
+int gca_reset(gca_cache_t* c) {
+    if (!c) return GCA_ERR_INVALID_ARG;
+    c->free_pages.clear();
+    for (int i = 0; i < c->num_pages; ++i) c->free_pages.insert(i);
+    c->image_pages.clear();
+    c->summary_pages.clear();
+    c->summary_opened_by.clear();
+    c->T = 0;
+    std::fill(c->layer_frames.begin(), c->layer_frames.end(), 0);
+    c->version += 1;
+    return GCA_OK;
+}
+
+int gca_get_layout(const gca_cache_t* c, int32_t F, gca_page_entry_t* out, int32_t cap, int32_t* n_out) {
+    if (!c || !n_out || cap < 0 || (cap > 0 && !out)) return GCA_ERR_INVALID_ARG;
+    if (F < 1 || F > c->T) return GCA_ERR_STATE;
+    std::vector<gca_page_entry_t> w;
+    if (!build_walk(c, F, w)) return GCA_ERR_STATE;
+    const int n = (int)w.size();
+    for (int i = 0; i < std::min(n, cap); ++i) out[i] = w[i];
+    *n_out = n;
+    return GCA_OK;
+}
+
+int gca_token_slot(const gca_cache_t* c, int32_t frame, int32_t tau, int32_t* page_id_out, int32_t* slot_out) {
+    if (!c || !page_id_out || !slot_out) return GCA_ERR_INVALID_ARG;
+    const int S = c->cfg.summary_tokens;
+    if (frame < 0 || frame >= c->T || tau < 0 || tau >= c->Lq) return GCA_ERR_INVALID_ARG;
+    if (tau < S) {
+        const long long idx = (long long)S * frame + tau;
+        *page_id_out = c->summary_pages[idx / c->P];
+        *slot_out = (int)(idx % c->P);
+        return GCA_OK;
+    }
+    auto it = c->image_pages.find(frame);
+    if (it == c->image_pages.end()) return GCA_ERR_STATE;
+    const int m = tau - S;
+    *page_id_out = it->second[m / c->P];
+    *slot_out = m % c->P;
+    return GCA_OK;
+}
+
+int gca_get_info(const gca_cache_t* c, gca_info_t* info) {
+    if (!c || !info) return GCA_ERR_INVALID_ARG;
+    info->num_pages = c->num_pages;
+    info->image_pages_per_frame = c->ipf;
+    info->frames = c->T;
+    info->full_frames = (int)c->image_pages.size();
+    info->resident_tokens = (long long)c->cfg.image_tokens * (long long)c->image_pages.size() +
+                            (long long)c->cfg.summary_tokens * c->T;
+    info->k_pool = c->kpool;
+    info->v_pool = c->vpool;
+    info->pool_bytes = c->pool_bytes;
+    info->scratch_bytes = c->ws_slots * kTileRows * (gca::kHeadDim + 1) * sizeof(float);
+    info->kernel_launches = c->launches;
+    return GCA_OK;
+}
+
+int gca_device_status(gca_cache_t* c, int32_t* status_out, int32_t clear) {
+    if (!c || !status_out) return GCA_ERR_INVALID_ARG;
+    *status_out = *(volatile int*)c->h_status;
+    if (clear) *(volatile int*)c->h_status = 0;
+    return GCA_OK;
+}
+
+int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* out, float* lse,
+               void* stream) {
+    if (!c || !q || !out) return GCA_ERR_INVALID_ARG;
+    const gca_config_t& g = c->cfg;
+    if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
+    if (F < 1 || F > g.max_query_frames) return GCA_ERR_INVALID_ARG;
+    if (F > c->T || c->layer_frames[layer] != c->T) return GCA_ERR_STATE;
+    if (int s = check_status(c)) return s;
+    DeviceGuard guard(c->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // walk list: rebuilt and uploaded when the page table or the block changed
+    if (c->up_version != c->version || c->up_F != F) {
+        std::vector<gca_page_entry_t> w;
+        if (!build_walk(c, F, w)) return GCA_ERR_STATE;
+        const int slot = c->ring_pos;
+        c->ring_pos = (c->ring_pos + 1) % kRing;
+        if (cudaEventSynchronize(c->stage_ev[slot]) != cudaSuccess) return GCA_ERR_CUDA;
+        WalkEntry* hs = c->h_stage[slot];
+        for (size_t i = 0; i < w.size(); ++i) {
+            const gca_page_entry_t& e = w[i];
+            hs[i] = make_int4(e.page_id, e.n_valid, e.first, e.kind == GCA_PAGE_IMAGE ? e.frame : -1);
+        }
+        if (cudaMemcpyAsync(c->d_walk, hs, sizeof(WalkEntry) * w.size(), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaEventRecord(c->stage_ev[slot], st) != cudaSuccess)
+            return GCA_ERR_CUDA;
+        c->up_version = c->version;
+        c->up_F = F;
+        c->up_n = (int)w.size();
+    }
+
+    const int R = F * c->Lq;
+    const size_t qbytes = (size_t)R * g.num_heads * gca::kHeadDim * c->elem;
+    const void* qd = q;
+    if (!is_device_ptr(q)) {
+        if (cudaMemcpyAsync(c->st_q, q, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        qd = c->st_q;
+    }
+    const bool out_host = !is_device_ptr(out);
+    const bool lse_host = lse && !is_device_ptr(lse);
+
+    gca::AttendParams p{};
+    p.walk = c->d_walk;
+    p.nwalk = c->up_n;
+    p.q = qd;
+    p.out = out_host ? c->st_out : out;
+    p.lse = lse ? (lse_host ? c->st_lse : lse) : nullptr;
+    p.R = R;
+    p.H = g.num_heads;
+    p.Lq = c->Lq;
+    p.first_query_frame = c->T - F;
+    p.rule = {g.num_anchor, g.window, g.summary_tokens, g.anchor_block ? 1 : 0};
+    p.scale = c->scale;
+    p.scale_log2 = c->scale * 1.4426950408889634f;
+    p.layer = layer;
+    p.num_pages = c->num_pages;
+    p.P = c->P;
+    p.status = c->d_status;
+    p.ws_o = c->ws_o;
+    p.ws_lse = c->ws_lse;
+
+    cudaError_t err;
+    if (g.dtype == GCA_DTYPE_BF16) {
+        // split: QT query tiles x W workers over the head-major page stream
+        p.QT = ceil_div(R, kTileRows);
+        const long long total = (long long)g.num_heads * p.nwalk;
+        long long w = std::max(1, c->sms / p.QT);
+        w = std::min<long long>(w, (total + 3) / 4);
+        w = std::max<long long>(w, 1);
+        p.seg = ceil_div(total, w);
+        p.W = ceil_div(total, p.seg);
+        bool need_merge = false;
+        for (int h = 0; h < g.num_heads && !need_merge; ++h)
+            need_merge = ((long long)h * p.nwalk) / p.seg != ((long long)(h + 1) * p.nwalk - 1) / p.seg;
+        err = gca::launch_attend_sm100(c->tmK, c->tmV, p, st);
+        c->launches += 1;
+        if (err == cudaSuccess && need_merge) {
+            err = gca::launch_merge(p, st);
+            c->launches += 1;
+        }
+    } else {
+        p.QT = ceil_div(R, kTileRows);
+        p.W = 1;
+        p.seg = 1;
+        err = gca::launch_attend_f32(p, c->kpool, c->vpool, st);
+        c->launches += 1;
+    }
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return GCA_ERR_CUDA;
+    }
+    if (out_host && cudaMemcpyAsync(out, c->st_out, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GCA_ERR_CUDA;
+    if (lse_host && cudaMemcpyAsync(lse, c->st_lse, (size_t)R * g.num_heads * sizeof(float),
+                                    cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GCA_ERR_CUDA;
+    return GCA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Internal declarations shared by the host code and the kernels of libgca.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gca {
+
+constexpr int kMaxImagePages = 128;     // image pages per frame (M <= 128 * P)
+constexpr int kHeadDim = 64;
+
+// Device walk-list entry: x = page id, y = tokens stored, z = first index
+// (image: among the frame's image tokens; summary: summary-stream index),
+// w = owning frame for an image page, -1 for a summary page.
+using WalkEntry = int4;
+
+// Visibility of one walk-list page to query frame i, as a prefix length: keys
+// 0..nvis-1 of the page are visible, the rest are not.  Every GCA mask is a
+// prefix of each page: an image page belongs to one frame and is all-or-none;
+// a summary page holds frames in stream order, so the visible tokens (frames
+// <= i) are its leading slots.
+struct MaskRule {
+    int n;             // anchor frames
+    int k;             // window frames (current frame included)
+    int S;             // summary tokens per frame
+    int anchor_block;  // anchors see each other in full
+};
+
+__host__ __device__ inline int visible_prefix(const MaskRule& r, int4 e, int i) {
+    if (e.w >= 0) {
+        const int j = e.w;
+        const bool vis = (r.anchor_block && i < r.n && j < r.n) ||
+                         (j <= i && (j < r.n || j >= i - r.k + 1));
+        return vis ? e.y : 0;
+    }
+    const int lim = (r.anchor_block && i < r.n) ? r.S * r.n : r.S * (i + 1);
+    int v = lim - e.z;
+    v = v < 0 ? 0 : v;
+    return v < e.y ? v : e.y;
+}
+
+struct AppendParams {
+    const void* k;            // [nlayers][Lq][H][D]
+    const void* v;
+    void* kpool;              // [L][num_pages][H][P][D]
+    void* vpool;
+    int layer0, nlayers;
+    int Lq, S, M, H, P, num_pages, elem_bytes;
+    int frame;
+    int sum_seq0;             // summary page sequence number of this frame's token 0
+    int sum_page[2];          // page ids of summary sequences sum_seq0, sum_seq0+1
+    int new_sum_seq;          // summary sequence opened by this frame, -1 if none
+    int img_pages[kMaxImagePages];
+};
+
+struct AttendParams {
+    const WalkEntry* walk;
+    int nwalk;
+    const void* q;            // [R][H][D]
+    void* out;                // [R][H][D]
+    float* lse;               // [R][H] natural log, nullable
+    int R, H, Lq;
+    int first_query_frame;    // frame of row 0
+    MaskRule rule;
+    float scale_log2;         // softmax scale * log2(e)
+    float scale;              // softmax scale
+    int layer, num_pages, P;
+    // split of the head-major (head, walk entry) stream over W workers
+    int QT, W, seg;
+    float* ws_o;              // [QT*(W+H-1)][128][D] partial outputs (normalised)
+    float* ws_lse;            // [QT*(W+H-1)][128] partial log2-sum-exp
+    int* status;              // device status word (host-mapped)
+};
+
+// launchers (return cudaError_t of the launch)
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
+                                const AttendParams& p, cudaStream_t s);
+cudaError_t launch_merge(const AttendParams& p, cudaStream_t s);
+cudaError_t launch_attend_f32(const AttendParams& p, const void* kpool, const void* vpool,
+                              cudaStream_t s);
+
+// device status codes
+enum : int {
+    kStatusWaitTimeout = 1,
+    kStatusBadPage = 2,
+};
+
+}  // namespace gca
