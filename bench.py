@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU seconds of the oracle sample")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the layer count (profiling captures of a smaller case)")
     return ap.parse_args()
 
 
@@ -222,6 +224,8 @@ def run_reference(args):
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = inputs.METRIC_518x378.with_(seed0=rank)
+    if args.layers:
+        w = w.with_(L=args.layers, name=f"{w.name}_layers{args.layers}")
     K, W = args.steps, args.warmup
     T_end = w.T
     n_pre = T_end - K - W

@@ -41,6 +41,7 @@ def test_tiny_stream_every_step(w):
     cache = gca.Cache.for_workload(w)
     sim = _sim(w)
     mirror = Mirror(w, [0])
+    errs = []
     for t in range(w.T):
         k = inputs.draw(w, t, "k").cuda()
         v = inputs.draw(w, t, "v").cuda()
@@ -55,9 +56,11 @@ def test_tiny_stream_every_step(w):
         out, lse = attend(cache, 0, q)
         want, wlse = oracle_step(mirror, 0, q.float().cpu().numpy(), t)
         torch.cuda.synchronize()
-        assert max_err(out, want) <= TOL[w.dtype], t
-        assert max_err(lse, wlse) <= LSE_TOL[w.dtype], t
+        errs.append((max_err(out, want), max_err(lse, wlse)))
+        assert errs[-1][0] <= TOL[w.dtype], t
+        assert errs[-1][1] <= LSE_TOL[w.dtype], t
     assert cache.status() == 0
+    print(f"{w.name}: max |dO| {max(e[0] for e in errs):.3e}, max |dlse| {max(e[1] for e in errs):.3e}")
 
 
 @pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
