@@ -67,6 +67,28 @@ def peaks():
         return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
 
 
+def rank_workload(rank: int, layers=None):
+    """The stream a rank runs: the metric workload seeded by the rank."""
+    w = inputs.METRIC_518x378.with_(seed0=rank)
+    if layers:
+        w = w.with_(L=layers, name=f"{w.name}_layers{layers}")
+    return w
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value over all ranks (time-like quantities: the job's time)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank: float, world: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: units all ranks processed / the max-over-ranks time."""
+    return units_per_rank * world / (elapsed_ms / 1e3)
+
+
 def lk_at(w, T):
     """Keys a single-frame query sees after T frames: M*min(T, n+k) + S*T."""
     return w.M * min(T, w.n + w.k) + w.S * T
@@ -223,9 +245,7 @@ def run_reference(args):
 
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
-    w = inputs.METRIC_518x378.with_(seed0=rank)
-    if args.layers:
-        w = w.with_(L=args.layers, name=f"{w.name}_layers{args.layers}")
+    w = rank_workload(rank, args.layers)
     K, W = args.steps, args.warmup
     T_end = w.T
     n_pre = T_end - K - W
@@ -331,25 +351,18 @@ def run_ours(args, rank, world, local_rank):
             hstep(j)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         fb = w.L * w.Lq * w.H * w.D * 2
-        e2e = {"value": E * w.L * world / (e2e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": job_value(E * w.L, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": 3 * fb, "d2h_bytes_per_step": fb}
 
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     if rank != 0:
         return
     pk = peaks()
     tr = traffic_record()
-    value = K * w.L * world / (elapsed_ms / 1e3)
+    value = job_value(K * w.L, world, elapsed_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",

@@ -8,27 +8,37 @@
 // page's visible keys are a prefix of its slots (see visible_prefix), so the
 // mask is one integer per (row, page).
 //
-// Work split.  Query rows form QT tiles of 128.  The head-major stream of
-// (head, walk entry) pairs is cut into W contiguous segments; CTA (qt, w)
-// runs query tile qt over segment w.  All QT tiles of a segment read the same
-// K/V pages in the same order at about the same time, so each page comes from
-// HBM once and from L2 for the other tiles.  A segment that covers a whole
-// head writes the final output; heads split between segments leave
-// normalised partials plus their log-sum-exp for the merge kernel.
+// Work split.  Query rows form pairs of 128-row tiles (256 rows per CTA).  The
+// head-major stream of (head, walk entry) pairs is cut into W contiguous
+// segments; CTA (pair, w) runs its two tiles over segment w.  All CTAs of a
+// segment read the same K/V pages in the same order at about the same time,
+// so each page comes from HBM once and from L2 for the others.  A segment that
+// covers a whole head writes the final output; heads split between segments
+// leave normalised partials plus their log-sum-exp for the merge kernel.
 //
-// Per CTA (192 threads, one CTA per SM):
-//   warps 0-3  softmax: thread t owns query row t of the tile (TMEM lane t);
-//              loads Q into TMEM, reads S rows from TMEM, online softmax in
-//              the log2 domain with a lazy rescale of O, writes P (bf16) into
-//              TMEM, final normalisation and store;
-//   warp 4     TMA producer: one (page, head) K tile and V tile per stage,
+// Per CTA (384 threads, one CTA per SM):
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread t owns query row t of
+//              its tile (TMEM lane t); loads Q into TMEM, reads S rows from
+//              TMEM, online softmax in the log2 domain with a lazy rescale of
+//              O, writes P (bf16) back over the S columns, final normalisation;
+//   warp 8     TMA producer: one (page, head) K tile and V tile per stage,
 //              128-byte swizzled boxes of P x 64 bf16, 4 stages;
-//   warp 5     MMA issuer (one thread) and TMEM owner:
-//                S_j  = Q K_j^T   tcgen05.mma kind::f16, A = Q from TMEM,
-//                                 B = K tile (K-major, SW128) from smem;
-//                O   += P_j V_j   A = P from TMEM, B = V tile (MN-major, SW128).
-// TMEM columns: S double buffer (2 x P), P double buffer (2 x P/2 packed
-// bf16x2), O (64), Q (32 packed) — 480 of 512 for P = 128.
+//   warp 9     MMA issuer (one thread) and TMEM owner (warps 10-11 idle).
+//              Per page j it issues
+//                S0 = Q0 K_j^T,  O1 += P1(j-1) V_{j-1},  S1 = Q1 K_j^T,
+//                O0 += P0(j) V_j
+//              so each softmax group overlaps the other group's two MMAs
+//              (A = Q or P from TMEM, B = K K-major / V MN-major from smem).
+// TMEM columns: S0, S1 (P aliased into their first P/2 columns), O0, O1, Q0,
+// Q1 — 448 of 512 for 128-token pages.  tcgen05 operations issued by one
+// thread execute in order, so S_t(j+1) is written only after PV_t(j) has read
+// P_t(j), and the commit after QK_t(j+1) also covers PV_t(j).
+//
+// Exponentials: scores are scaled and shifted with packed f32x2 FMAs; part of
+// each row's 2^x runs on the MUFU unit (ex2.approx) and part on the FMA pipe
+// as a degree-3 minimax polynomial after round-to-nearest range reduction
+// (coefficients from exp2_poly_fit.py), so that neither pipe alone bounds the
+// softmax.
 //
 // Every wait on an mbarrier is bounded by a %globaltimer deadline; on expiry
 // the thread raises the CTA abort flag and the device status word, every role
@@ -42,24 +52,42 @@ namespace gca {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kWarpTMA = 4;
-constexpr int kWarpMMA = 5;
-constexpr int kStages = 4;
+constexpr int kThreads = 384;               // 3 warpgroups: softmax 0, softmax 1, TMA + MMA
+constexpr int kWarpTMA = 8;
+constexpr int kWarpMMA = 9;
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
+// the two softmax warpgroups take 208, the producer warpgroup keeps 80:
+// 256 x 208 + 128 x 80 = 63488 <= 64512.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsProducer = 80;
+static_assert(256 * kRegsSoftmax + 128 * kRegsProducer <= kThreads * 168, "register split");
+#ifndef GCA_ATTEND_STAGES
+#define GCA_ATTEND_STAGES 4
+#endif
+#ifndef GCA_POLY_PAIRS
+#define GCA_POLY_PAIRS 6
+#endif
+constexpr int kStages = GCA_ATTEND_STAGES;
 constexpr int kRows = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
+constexpr int kPolyPairs = GCA_POLY_PAIRS;  // of each 16 column pairs, this many use the FMA-pipe 2^x
+
+// 2^f on [-1/2, 1/2], minimax relative error 7.5e-5 (exp2_poly_fit.py)
+constexpr float kExpC0 = 0x1.fff692p-1f;
+constexpr float kExpC1 = 0x1.62f31ap-1f;
+constexpr float kExpC2 = 0x1.f0de1ap-3f;
+constexpr float kExpC3 = 0x1.c3f76p-5f;
 
 template <int PAGE>
 struct Layout {
     static constexpr int kTileBytes = PAGE * 128;          // PAGE x 64 bf16
     static constexpr int kStageBytes = 2 * kTileBytes;     // K then V
-    static constexpr int kColS = 0;                        // + buffer * PAGE
-    static constexpr int kColP = 2 * PAGE;                 // + buffer * PAGE/2
-    static constexpr int kColO = 3 * PAGE;
-    static constexpr int kColQ = 3 * PAGE + 64;
-    static_assert(kColQ + 32 <= (int)kTmemCols, "TMEM budget");
+    static constexpr int kColS = 0;                        // + tile * PAGE (P in the first PAGE/2)
+    static constexpr int kColO = 2 * PAGE;                 // + tile * 64
+    static constexpr int kColQ = 2 * PAGE + 128;           // + tile * 32
+    static_assert(kColQ + 64 <= (int)kTmemCols, "TMEM budget");
     static constexpr int kNumBars = 2 * kStages + 9;
     static constexpr int kSmemBytes = kStages * kStageBytes + kNumBars * 8 + 16 + 1024;
 };
@@ -102,7 +130,7 @@ struct Ctl {
 };
 
 // Bounded parity wait.  honour_abort = false is used while draining.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, bool honour_abort = true) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, bool honour_abort = true) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
@@ -213,6 +241,57 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+
+// packed f32x2 arithmetic (two lanes of work per instruction)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unf2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for two values on the FMA pipe: x = j + f, j = rne(x) through the
+// 1.5*2^23 shifter, p(f) by Horner, then j added to the exponent field.
+// x is clamped to >= -125 so the exponent never underflows into the sign.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    const uint64_t x = f2(x0, x1);
+    const uint64_t t = fadd2(x, f2(12582912.f, 12582912.f));
+    const uint64_t j = fadd2(t, f2(-12582912.f, -12582912.f));
+    const uint64_t f = ffma2(j, f2(-1.f, -1.f), x);
+    uint64_t p = ffma2(f2(kExpC3, kExpC3), f, f2(kExpC2, kExpC2));
+    p = ffma2(p, f, f2(kExpC1, kExpC1));
+    p = ffma2(p, f, f2(kExpC0, kExpC0));
+    float t0, t1, p0, p1;
+    unf2(t, t0, t1);
+    unf2(p, p0, p1);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -229,11 +308,10 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const uint32_t bar0 = smem_u32(bars);
     auto kv_full = [&](int s) { return bar0 + 8u * s; };
     auto kv_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto s_full = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
-    auto s_free = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
-    const uint32_t p_full = bar0 + 8u * (2 * kStages + 4);
-    auto pv_done = [&](int b) { return bar0 + 8u * (2 * kStages + 5 + b); };
-    const uint32_t q_ready = bar0 + 8u * (2 * kStages + 7);
+    auto s_full = [&](int t) { return bar0 + 8u * (2 * kStages + t); };
+    auto p_full = [&](int t) { return bar0 + 8u * (2 * kStages + 2 + t); };
+    auto pv_done = [&](int t) { return bar0 + 8u * (2 * kStages + 4 + t); };
+    auto q_ready = [&](int t) { return bar0 + 8u * (2 * kStages + 6 + t); };
     const uint32_t drain = bar0 + 8u * (2 * kStages + 8);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -241,8 +319,8 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qt = blockIdx.x;
-    const int w = blockIdx.y;
+    const int qp = blockIdx.x;                 // pair of 128-row query tiles
+    const int w = blockIdx.y;                  // worker (segment of the page stream)
     const long long total = (long long)p.H * p.nwalk;
     const long long g0 = (long long)w * p.seg;
     const long long g1 = (g0 + p.seg < total) ? g0 + p.seg : total;
@@ -253,13 +331,12 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             mbar_init(kv_full(s), 1);
             mbar_init(kv_empty(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(s_full(b), 1);
-            mbar_init(s_free(b), kRows);
-            mbar_init(pv_done(b), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full(t), 1);
+            mbar_init(p_full(t), kRows);
+            mbar_init(pv_done(t), 1);
+            mbar_init(q_ready(t), kRows);
         }
-        mbar_init(p_full, kRows);
-        mbar_init(q_ready, kRows);
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -280,13 +357,14 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     __syncthreads();
     fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == kWarpTMA) {
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+      if (warp == kWarpTMA) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int issued = 0;
             bool ok = true;
-            for (int j = 0; j < J && ok; ++j) {
+            for (int j = 0; j < J; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages && !wait_bar(kv_empty(st), ((j / kStages) - 1) & 1, ctl)) {
                     ok = false;
@@ -322,65 +400,68 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_bf16(kRows, PAGE, false);
             constexpr uint32_t kIdescPV = idesc_bf16(kRows, 64, true);
-            bool ok = true;
-            auto issue_pv = [&](int jj) -> bool {
-                if (!wait_bar(p_full, jj & 1, ctl)) return false;
-                fence_after();
-                const int st = jj % kStages;
-                const uint32_t vaddr = sbase + st * L::kStageBytes + L::kTileBytes;
-                const bool first = (jj == 0) || ((g0 + jj) % p.nwalk == 0);
-                const uint32_t pcol = tmem + L::kColP + (jj & 1) * (PAGE / 2);
+            auto qk = [&](int t, int j) {
+                const uint32_t kaddr = sbase + (j % kStages) * L::kStageBytes;
+                const uint32_t scol = tmem + L::kColS + t * PAGE;
 #pragma unroll
-                for (int kk = 0; kk < PAGE / 16; ++kk) {
-                    // 16 keys per step: P columns 8kk..8kk+7, V rows 16kk..16kk+15
-                    mma_ts(tmem + L::kColO, pcol + kk * 8,
+                for (int kk = 0; kk < 4; ++kk)   // 16 head dims per step
+                    mma_ts(scol, tmem + L::kColQ + t * 32 + kk * 8,
+                           desc_sw128(kaddr + kk * 32, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                mma_commit(s_full(t));
+            };
+            auto pv = [&](int t, int j) -> bool {
+                if (!wait_bar(p_full(t), j & 1, ctl)) return false;
+                fence_after();
+                const int st = j % kStages;
+                const uint32_t vaddr = sbase + st * L::kStageBytes + L::kTileBytes;
+                const bool first = (j == 0) || ((g0 + j) % p.nwalk == 0);
+                const uint32_t pcol = tmem + L::kColS + t * PAGE;
+#pragma unroll
+                for (int kk = 0; kk < PAGE / 16; ++kk)   // 16 keys per step
+                    mma_ts(tmem + L::kColO + t * 64, pcol + kk * 8,
                            desc_sw128(vaddr + kk * 2048, L::kTileBytes, 1024), kIdescPV,
                            (first && kk == 0) ? 0u : 1u);
-                }
-                mma_commit(kv_empty(st));
-                mma_commit(pv_done(jj & 1));
+                mma_commit(pv_done(t));
+                if (t == 1) mma_commit(kv_empty(st));
                 return true;
             };
+            bool ok = true;
             int sidx = 0;
             for (int j = 0; j < J; ++j) {
                 const bool seg_first = (j == 0) || ((g0 + j) % p.nwalk == 0);
-                if (seg_first) {
-                    if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
-                    if (!wait_bar(q_ready, sidx & 1, ctl)) { ok = false; break; }
-                    ++sidx;
-                }
-                const int st = j % kStages;
-                if (!wait_bar(kv_full(st), (j / kStages) & 1, ctl)) { ok = false; break; }
-                if (j >= 2 && !wait_bar(s_free(j & 1), ((j >> 1) - 1) & 1, ctl)) { ok = false; break; }
+                if (seg_first && !wait_bar(q_ready(0), sidx & 1, ctl)) { ok = false; break; }
+                if (!wait_bar(kv_full(j % kStages), (j / kStages) & 1, ctl)) { ok = false; break; }
                 fence_after();
-                const uint32_t kaddr = sbase + st * L::kStageBytes;
-                const uint32_t scol = tmem + L::kColS + (j & 1) * PAGE;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    // 16 head dims per step: Q columns 8kk..8kk+7, K bytes 32kk..32kk+31 of each row
-                    mma_ts(scol, tmem + L::kColQ + kk * 8, desc_sw128(kaddr + kk * 32, 16, 1024),
-                           kIdescQK, kk > 0 ? 1u : 0u);
+                qk(0, j);
+                if (j > 0 && !pv(1, j - 1)) { ok = false; break; }
+                if (seg_first) {
+                    if (!wait_bar(q_ready(1), sidx & 1, ctl)) { ok = false; break; }
+                    ++sidx;
+                    fence_after();
                 }
-                mma_commit(s_full(j & 1));
-                if (!seg_first && !issue_pv(j - 1)) { ok = false; break; }
+                qk(1, j);
+                if (!pv(0, j)) { ok = false; break; }
             }
-            if (ok) issue_pv(J - 1);
+            if (ok) pv(1, J - 1);
             // drain: every MMA issued above completes before TMEM is released
             mma_commit(drain);
             wait_bar(drain, 0, ctl, false);
         }
         __syncwarp();
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ------------------------------------------------------------ softmax
-        const int rl = threadIdx.x;                    // row in the tile, TMEM lane
-        const int row = qt * kRows + rl;
+        const int t = warp >> 2;                       // query tile of this warp group
+        const int quarter = warp & 3;
+        const int rl = quarter * 32 + lane;            // row in the tile, TMEM lane
+        const int row = (qp * 2 + t) * kRows + rl;
         const bool valid = row < p.R;
         const int qframe = p.first_query_frame + (valid ? row / p.Lq : 0);
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t t_s = tmem + lane_base + L::kColS;
-        const uint32_t t_p = tmem + lane_base + L::kColP;
-        const uint32_t t_o = tmem + lane_base + L::kColO;
-        const uint32_t t_q = tmem + lane_base + L::kColQ;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + L::kColS + t * PAGE;
+        const uint32_t t_o = tmem + lane_base + L::kColO + t * 64;
+        const uint32_t t_q = tmem + lane_base + L::kColQ + t * 32;
         const float sl2 = p.scale_log2;
         const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
 
@@ -403,7 +484,7 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             tmem_st32(t_q, r);
             tmem_wait_st();
             fence_before();
-            mbar_arrive(q_ready);
+            mbar_arrive(q_ready(t));
         };
         auto all_ok = [&](bool ok) { return __all_sync(0xffffffffu, ok); };
 
@@ -422,22 +503,35 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             const int4 ent = __ldg(&p.walk[e]);
             const int nvis = visible_prefix(p.rule, ent, qframe);
 
-            if (!all_ok(wait_bar(s_full(j & 1), (j >> 1) & 1, ctl))) break;
+            // S_t(j) is complete, and so is PV_t(j-1) (one commit covers both)
+            if (!all_ok(wait_bar(s_full(t), j & 1, ctl))) break;
             fence_after();
-            uint32_t sr[PAGE];
+            uint32_t r[PAGE];
 #pragma unroll
-            for (int c = 0; c < PAGE / 32; ++c) tmem_ld32(t_s + (j & 1) * PAGE + 32 * c, sr + 32 * c);
+            for (int c = 0; c < PAGE / 32; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
             tmem_wait_ld();
-            fence_before();
-            mbar_arrive(s_free(j & 1));
-
-            float s[PAGE];
-            float mx = -INFINITY;
+            if (nvis < PAGE) {
 #pragma unroll
-            for (int c = 0; c < PAGE; ++c) {
-                s[c] = (c < nvis) ? __uint_as_float(sr[c]) : -INFINITY;
-                mx = fmaxf(mx, s[c]);
+                for (int c = 0; c < PAGE; ++c) r[c] = (c < nvis) ? r[c] : 0xff800000u;
             }
+            // row max: 16 independent three-input max chains, then a tree
+            float acc[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(r[i]);
+#pragma unroll
+            for (int c = 16; c + 32 <= PAGE; c += 32)
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc[i] = fmax3(acc[i], __uint_as_float(r[c + i]), __uint_as_float(r[c + 16 + i]));
+            if constexpr ((PAGE - 16) % 32 != 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = fmaxf(acc[i], __uint_as_float(r[PAGE - 16 + i]));
+            }
+            const float a0 = fmax3(acc[0], acc[1], acc[2]), a1 = fmax3(acc[3], acc[4], acc[5]);
+            const float a2 = fmax3(acc[6], acc[7], acc[8]), a3 = fmax3(acc[9], acc[10], acc[11]);
+            const float a4 = fmax3(acc[12], acc[13], acc[14]);
+            const float mx = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, acc[15]), -INFINITY);
+
             const float mt = mx * sl2;
             float alpha = 1.f;
             bool resc = false;
@@ -450,42 +544,62 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             }
             const float msub = (m_run == -INFINITY) ? 0.f : m_run;
 
-            // P buffer (j & 1) was last read by PV_{j-2}
-            if (j >= 2 && !all_ok(wait_bar(pv_done(j & 1), ((j - 2) >> 1) & 1, ctl))) break;
-            float rs = 0.f;
+            if (__any_sync(0xffffffffu, resc)) {
+                // PV_t(j-1) has completed (covered by the s_full commit)
+                const uint64_t a2v = f2(alpha, alpha);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t o[32];
+                    tmem_ld32(t_o + 32 * half, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int d = 0; d < 32; d += 2) {
+                        float x0, x1;
+                        unf2(fmul2(f2(__uint_as_float(o[d]), __uint_as_float(o[d + 1])), a2v), x0, x1);
+                        o[d] = __float_as_uint(x0);
+                        o[d + 1] = __float_as_uint(x1);
+                    }
+                    tmem_st32(t_o + 32 * half, o);
+                }
+            }
+
+            // P = 2^(s * scale_log2 - m), packed bf16, written over the S columns
+            const uint64_t sl2v = f2(sl2, sl2);
+            const uint64_t nmv = f2(-msub, -msub);
+            uint64_t rs2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < PAGE / 32; ++c) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, -msub));
-                    const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, -msub));
-                    rs += p0 + p1;
+                    const uint64_t x = ffma2(f2(__uint_as_float(r[32 * c + 2 * i]),
+                                                __uint_as_float(r[32 * c + 2 * i + 1])),
+                                             sl2v, nmv);
+                    float x0, x1, p0, p1;
+                    unf2(x, x0, x1);
+                    if (i < kPolyPairs) {
+                        exp2_poly2(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    }
+                    rs2[i & 3] = fadd2(rs2[i & 3], f2(p0, p1));
                     pk[i] = pack_bf16(p0, p1);
                 }
-                tmem_st16(t_p + (j & 1) * (PAGE / 2) + 16 * c, pk);
+                tmem_st16(t_s + 16 * c, pk);
             }
-            l_run = l_run * alpha + rs;
-
-            if (__any_sync(0xffffffffu, resc)) {
-                // O must hold PV_{j-1} before it is rescaled
-                if (!all_ok(wait_bar(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, ctl))) break;
-                fence_after();
-                uint32_t o[64];
-                tmem_ld32(t_o, o);
-                tmem_ld32(t_o + 32, o + 32);
-                tmem_wait_ld();
-#pragma unroll
-                for (int d = 0; d < 64; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * alpha);
-                tmem_st32(t_o, o);
-                tmem_st32(t_o + 32, o + 32);
-            }
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            unf2(rs2[0], s0, s1);
+            unf2(rs2[1], s2, s3);
+            unf2(rs2[2], s4, s5);
+            unf2(rs2[3], s6, s7);
+            l_run = l_run * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
             tmem_wait_st();
             fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(p_full(t));
 
             if (seg_last) {
-                if (!all_ok(wait_bar(pv_done(j & 1), (j >> 1) & 1, ctl))) break;
+                if (!all_ok(wait_bar(pv_done(t), j & 1, ctl))) break;
                 fence_after();
                 uint32_t o[64];
                 tmem_ld32(t_o, o);
@@ -510,8 +624,8 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         }
                         if (p.lse) p.lse[(long long)row * p.H + h] = lse2 * 0.69314718055994531f;
                     }
-                } else {
-                    const long long slot = (long long)qt * (p.W + p.H - 1) + w + h;
+                } else if (valid) {
+                    const long long slot = (long long)(qp * 2 + t) * (p.W + p.H - 1) + w + h;
                     float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kRows + rl) * 64);
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
@@ -588,7 +702,7 @@ cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const Atte
     cudaError_t e = cudaFuncSetAttribute(attend_kernel<PAGE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.QT, p.W);
+    dim3 grid((p.QT + 1) / 2, p.W);
     attend_kernel<PAGE><<<grid, kThreads, smem, s>>>(tk, tv, p);
     return cudaGetLastError();
 }

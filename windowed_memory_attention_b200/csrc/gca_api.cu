@@ -248,10 +248,11 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
         ok = cudaHostAlloc((void**)&c->h_stage[i], sizeof(WalkEntry) * c->walk_cap, cudaHostAllocDefault) == cudaSuccess &&
              cudaEventCreateWithFlags(&c->stage_ev[i], cudaEventDisableTiming) == cudaSuccess;
     }
-    // split-KV scratch: per query tile at most W + H - 1 (worker, head) partials,
-    // with QT * W <= max(SMs, QT)
+    // split-KV scratch: per 128-row query tile at most W + H - 1 (worker, head)
+    // partials; W <= max(1, SMs / tile pairs), so QT * W <= 2 * max(SMs, pairs)
     const int qt_max = ceil_div((long long)g.max_query_frames * c->Lq, kTileRows);
-    c->ws_slots = (size_t)std::max(c->sms, qt_max) + (size_t)qt_max * (g.num_heads - 1);
+    const int qp_max = (qt_max + 1) / 2;
+    c->ws_slots = 2 * (size_t)std::max(c->sms, qp_max) + (size_t)qt_max * (g.num_heads - 1);
     if (g.dtype == GCA_DTYPE_BF16) {
         ok = ok && cudaMalloc(&c->ws_o, c->ws_slots * kTileRows * gca::kHeadDim * sizeof(float)) == cudaSuccess &&
              cudaMalloc(&c->ws_lse, c->ws_slots * kTileRows * sizeof(float)) == cudaSuccess;
@@ -528,7 +529,7 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
         // split: QT query tiles x W workers over the head-major page stream
         p.QT = ceil_div(R, kTileRows);
         const long long total = (long long)g.num_heads * p.nwalk;
-        long long w = std::max(1, c->sms / p.QT);
+        long long w = std::max(1, c->sms / ((p.QT + 1) / 2));   // CTAs = tile pairs x workers
         w = std::min<long long>(w, (total + 3) / 4);
         w = std::max<long long>(w, 1);
         p.seg = ceil_div(total, w);
