@@ -37,40 +37,43 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     char* pool = static_cast<char*>(tensor ? p.vpool : p.kpool);
 
     const int row_bytes = kHeadDim * p.elem_bytes;       // one token of one head
-    const int cpr = row_bytes >> 4;                      // 16-byte chunks per row
+    const int cpr_shift = p.elem_bytes == 2 ? 3 : 4;     // 16-byte chunks per row: 8 or 16
+    const unsigned cpr = 1u << cpr_shift;
     const long long tile_bytes = (long long)p.P * row_bytes;
     const long long layer_src = (long long)p.Lq * p.H * row_bytes;
     src += (long long)ll * layer_src;
     char* lpool = pool + (long long)layer * p.num_pages * p.H * tile_bytes;
 
-    const long long n_copy = (long long)p.Lq * p.H * cpr;
+    // 32-bit index arithmetic: one (layer, tensor) has at most Lq*H*16 chunks
+    const unsigned H = (unsigned)p.H;
+    const unsigned n_copy = (unsigned)p.Lq * H * cpr;
     // zero regions, per head: image tail slots and new summary page tail
-    const int img_tail = (p.M % p.P) ? (p.P - p.M % p.P) : 0;
-    int sum_from = 0, sum_tail = 0;
+    const unsigned img_tail = (p.M % p.P) ? (unsigned)(p.P - p.M % p.P) : 0u;
+    unsigned sum_from = 0, sum_tail = 0;
     if (p.new_sum_seq >= 0) {
-        sum_from = p.S * (p.frame + 1) - p.new_sum_seq * p.P;   // first unused slot
-        sum_tail = p.P - sum_from;
+        sum_from = (unsigned)(p.S * (p.frame + 1) - p.new_sum_seq * p.P);   // first unused slot
+        sum_tail = (unsigned)p.P - sum_from;
     }
-    const long long n_zimg = (long long)p.H * img_tail * cpr;
-    const long long n_zsum = (long long)p.H * sum_tail * cpr;
-    const long long total = n_copy + n_zimg + n_zsum;
+    const unsigned n_zimg = H * img_tail * cpr;
+    const unsigned n_zsum = H * sum_tail * cpr;
+    const unsigned total = n_copy + n_zimg + n_zsum;
 
     // destination of chunk u (and whether it is a zero fill)
-    auto dest = [&](long long u, bool& zero) -> char* {
+    auto dest = [&](unsigned u, bool& zero) -> char* {
         if (u < n_copy) {
             zero = false;
-            const int chunk = (int)(u % cpr);
-            const long long th = u / cpr;
-            const int h = (int)(th % p.H);
-            const int tau = (int)(th / p.H);
+            const unsigned chunk = u & (cpr - 1);
+            const unsigned th = u >> cpr_shift;
+            const unsigned tau = th / H;
+            const unsigned h = th - tau * H;
             int page, slot;
-            if (tau < p.S) {
-                const int idx = p.S * p.frame + tau;
+            if ((int)tau < p.S) {
+                const int idx = p.S * p.frame + (int)tau;
                 const int seq = idx / p.P;
                 page = p.sum_page[seq - p.sum_seq0];
                 slot = idx - seq * p.P;
             } else {
-                const int m = tau - p.S;
+                const int m = (int)tau - p.S;
                 const int seq = m / p.P;
                 page = p.img_pages[seq];
                 slot = m - seq * p.P;
@@ -79,11 +82,12 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
                    (long long)slot * row_bytes + chunk * 16;
         }
         zero = true;
-        long long z = u - n_copy;
-        int page, slot0, nslots;
+        unsigned z = u - n_copy;
+        int page;
+        unsigned slot0, nslots;
         if (z < n_zimg) {
             page = p.img_pages[(p.M - 1) / p.P];
-            slot0 = p.P - img_tail;
+            slot0 = (unsigned)p.P - img_tail;
             nslots = img_tail;
         } else {
             z -= n_zimg;
@@ -91,25 +95,24 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
             slot0 = sum_from;
             nslots = sum_tail;
         }
-        const int chunk = (int)(z % cpr);
-        const long long ts = z / cpr;
-        const int sl = (int)(ts % nslots);
-        const int h = (int)(ts / nslots);
+        const unsigned chunk = z & (cpr - 1);
+        const unsigned ts = z >> cpr_shift;
+        const unsigned h = ts / nslots;
+        const unsigned sl = ts - h * nslots;
         return lpool + ((long long)page * p.H + h) * tile_bytes +
                (long long)(slot0 + sl) * row_bytes + chunk * 16;
     };
 
     // four independent chunks per thread per iteration: loads first, then stores
     constexpr int U = 4;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long base = (long long)blockIdx.x * blockDim.x + threadIdx.x; base < total;
-         base += U * stride) {
+    const unsigned stride = gridDim.x * blockDim.x;
+    for (unsigned base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += U * stride) {
         int4 val[U];
         char* dst[U];
         bool zero[U];
 #pragma unroll
         for (int i = 0; i < U; ++i) {
-            const long long u = base + i * stride;
+            const unsigned u = base + i * stride;
             dst[i] = nullptr;
             if (u < total) {
                 dst[i] = dest(u, zero[i]);
@@ -126,9 +129,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 }  // namespace
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = p.sms > 0 ? p.sms : 148;
     const long long per_lt = (long long)p.Lq * p.H * (kHeadDim * p.elem_bytes / 16);
     // about 4 chunks per thread per (layer, tensor), at most 8 blocks per SM overall
     long long want = (per_lt + 256 * 4 - 1) / (256 * 4);

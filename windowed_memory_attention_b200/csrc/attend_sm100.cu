@@ -490,6 +490,8 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 
         float m_run = -INFINITY, l_run = 0.f;
         load_q((int)(g0 / p.nwalk));
+        // walk entries are read one page ahead, off the critical path
+        int4 ent_next = __ldg(&p.walk[(int)(g0 % p.nwalk)]);
         for (int j = 0; j < J; ++j) {
             const long long g = g0 + j;
             const int h = (int)(g / p.nwalk);
@@ -500,7 +502,8 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 m_run = -INFINITY;
                 l_run = 0.f;
             }
-            const int4 ent = __ldg(&p.walk[e]);
+            const int4 ent = ent_next;
+            if (j + 1 < J) ent_next = __ldg(&p.walk[e + 1 == p.nwalk ? 0 : e + 1]);
             const int nvis = visible_prefix(p.rule, ent, qframe);
 
             // S_t(j) is complete, and so is PV_t(j-1) (one commit covers both)

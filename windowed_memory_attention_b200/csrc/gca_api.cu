@@ -359,6 +359,7 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
     p.P = c->P;
     p.num_pages = c->num_pages;
     p.elem_bytes = (int)c->elem;
+    p.sms = c->sms;
     p.frame = t;
     const int S = g.summary_tokens;
     p.sum_seq0 = (S * t) / c->P;

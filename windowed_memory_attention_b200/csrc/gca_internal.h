@@ -52,6 +52,7 @@ struct AppendParams {
     int sum_page[2];          // page ids of summary sequences sum_seq0, sum_seq0+1
     int new_sum_seq;          // summary sequence opened by this frame, -1 if none
     int img_pages[kMaxImagePages];
+    int sms;                  // SMs of the device (grid sizing)
 };
 
 struct AttendParams {
