@@ -190,6 +190,29 @@ int gca_device_status(gca_cache_t* cache, int32_t* status_out, int32_t clear);
 /* Static text of a status code. */
 const char* gca_status_string(int status);
 
+/* GCA attention over caller-owned pages, allocating no device memory.  The
+ * paper has no counterpart; it serves callers that cannot call cudaMalloc:
+ * a host framework whose caching allocator owns the device memory, or a
+ * real-time loop that must not make a call that can synchronise the device.
+ * Computes what gca_attend computes, with the bf16 tcgen05 kernel, for pools
+ * k_pool/v_pool laid out [num_layers][num_pages][num_heads][page_size][64]
+ * bf16 (device), a walk list of nwalk gca_page_entry_t (host or device; the
+ * entries gca_get_layout returns), q/out [F][tokens_per_frame][H][64] bf16
+ * (device) whose row 0 belongs to frame first_query_frame, lse [F][Lq][H]
+ * float32 (device, nullable) and status (device int, nullable: raised like
+ * the cache's status word).  Scratch lives in one static device array of
+ * 18 MiB per GPU: at most 32768 walk entries and 512 partial tiles of 128
+ * query rows (ceil(F*Lq/128) * H <= 512), else GCA_ERR_CAPACITY.  The first
+ * call on a device looks up the array's address (call it before any stream
+ * capture); calls whose GPU work overlaps share the array and race. */
+int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, int32_t num_layers,
+                             int32_t num_pages, int32_t num_heads, int32_t page_size,
+                             int32_t layer, const gca_page_entry_t* walk, int32_t nwalk,
+                             const void* q, int32_t num_query_frames, int32_t tokens_per_frame,
+                             int32_t first_query_frame, int32_t num_anchor, int32_t window,
+                             int32_t summary_tokens, int32_t anchor_block, float softmax_scale,
+                             void* out, float* lse, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

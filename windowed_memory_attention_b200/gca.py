@@ -24,7 +24,7 @@ STATUS = {0: "GCA_OK", 1: "GCA_ERR_INVALID_ARG", 2: "GCA_ERR_CAPACITY", 3: "GCA_
           4: "GCA_ERR_UNSUPPORTED", 5: "GCA_ERR_CUDA", 6: "GCA_ERR_DEVICE_CHECK"}
 EXPORTS = ("gca_cache_create", "gca_cache_destroy", "gca_append_frame", "gca_evict_to_summary",
            "gca_attend", "gca_reset", "gca_get_layout", "gca_token_slot", "gca_get_info",
-           "gca_device_status", "gca_status_string")
+           "gca_device_status", "gca_status_string", "gca_attend_pages_noalloc")
 
 
 class gca_config_t(ctypes.Structure):
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "gca_token_slot": [vp, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
             "gca_get_info": [vp, ctypes.POINTER(gca_info_t)],
             "gca_device_status": [vp, ctypes.POINTER(i32), i32],
+            "gca_attend_pages_noalloc": [vp, vp, i32, i32, i32, i32, i32, vp, i32, vp, i32, i32,
+                                         i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -179,6 +181,22 @@ def gca_device_status(cache, clear: bool = False) -> int:
     s = ctypes.c_int32(0)
     _check("gca_device_status", lib().gca_device_status(cache, ctypes.byref(s), int(clear)))
     return s.value
+
+
+def gca_attend_pages_noalloc(k_pool, v_pool, *, num_layers: int, num_pages: int, num_heads: int,
+                             page_size: int, layer: int, walk, nwalk: int, q: torch.Tensor,
+                             num_query_frames: int, tokens_per_frame: int, first_query_frame: int,
+                             num_anchor: int, window: int, summary_tokens: int,
+                             anchor_block: bool, softmax_scale: float, out: torch.Tensor,
+                             lse: Optional[torch.Tensor] = None, status=None, stream=None) -> None:
+    """Attention over caller-owned pools with no device allocation (see gca.h).
+    ``walk`` is a ctypes array of gca_page_entry_t or a device pointer."""
+    _check("gca_attend_pages_noalloc", lib().gca_attend_pages_noalloc(
+        ctypes.c_void_p(k_pool), ctypes.c_void_p(v_pool), num_layers, num_pages, num_heads,
+        page_size, layer, walk if not isinstance(walk, int) else ctypes.c_void_p(walk), nwalk,
+        _ptr(q), num_query_frames, tokens_per_frame, first_query_frame, num_anchor, window,
+        summary_tokens, int(bool(anchor_block)), softmax_scale, _ptr(out), _ptr(lse),
+        _ptr(status), _stream(stream)))
 
 
 class Cache:
