@@ -19,8 +19,8 @@
 // Per CTA (384 threads, one CTA per SM):
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread t owns query row t of
 //              its tile (TMEM lane t); loads Q into TMEM, reads S rows from
-//              TMEM, online softmax in the log2 domain with a lazy rescale of
-//              O, writes P (bf16) back over the S columns, final normalisation;
+//              TMEM, online softmax in the log2 domain, writes P (bf16) back
+//              over the S columns, final normalisation;
 //   warp 8     TMA producer: one (page, head) K tile and V tile per stage,
 //              128-byte swizzled boxes of P x 64 bf16, 4 stages;
 //   warp 9     MMA issuer (one thread) and TMEM owner (warps 10-11 idle).
@@ -34,11 +34,15 @@
 // thread execute in order, so S_t(j+1) is written only after PV_t(j) has read
 // P_t(j), and the commit after QK_t(j+1) also covers PV_t(j).
 //
-// Exponentials: scores are scaled and shifted with packed f32x2 FMAs; part of
-// each row's 2^x runs on the MUFU unit (ex2.approx) and part on the FMA pipe
-// as a degree-3 minimax polynomial after round-to-nearest range reduction
-// (coefficients from exp2_poly_fit.py), so that neither pipe alone bounds the
-// softmax.
+// Softmax: a page is exponentiated against the row's running max without
+// computing the page max first.  Since relative precision does not depend on
+// scale, values up to 2^64 are as good as values up to 1; a row whose page
+// sum reaches 2^64 (or overflows) takes the exact path instead: page max, O
+// rescaled by 2^(m_old - m_new), exponentials recomputed.  The first page of
+// every head always takes the exact path.  Scores are scaled and shifted with
+// packed f32x2 FMAs; two of every sixteen column pairs get 2^x from a
+// degree-3 minimax polynomial on the FMA pipe (exp2_poly_fit.py), the rest
+// from the MUFU unit (ex2.approx).
 //
 // Every wait on an mbarrier is bounded by a %globaltimer deadline; on expiry
 // the thread raises the CTA abort flag and the device status word, every role
@@ -56,22 +60,21 @@ constexpr int kThreads = 384;               // 3 warpgroups: softmax 0, softmax 
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
-// the two softmax warpgroups take 208, the producer warpgroup keeps 80:
-// 256 x 208 + 128 x 80 = 63488 <= 64512.
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsProducer = 80;
+// the two softmax warpgroups take 216, the producer warpgroup keeps 64:
+// 256 x 216 + 128 x 64 = 63488 <= 64512.
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsProducer = 64;
 static_assert(256 * kRegsSoftmax + 128 * kRegsProducer <= kThreads * 168, "register split");
 #ifndef GCA_ATTEND_STAGES
 #define GCA_ATTEND_STAGES 4
 #endif
 #ifndef GCA_POLY_PAIRS
-#define GCA_POLY_PAIRS 6
+#define GCA_POLY_PAIRS 2
 #endif
 constexpr int kStages = GCA_ATTEND_STAGES;
 constexpr int kRows = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
 constexpr int kPolyPairs = GCA_POLY_PAIRS;  // of each 16 column pairs, this many use the FMA-pipe 2^x
 
 // 2^f on [-1/2, 1/2], minimax relative error 7.5e-5 (exp2_poly_fit.py)
@@ -325,6 +328,9 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const long long g0 = (long long)w * p.seg;
     const long long g1 = (g0 + p.seg < total) ? g0 + p.seg : total;
     const int J = (int)(g1 - g0);
+    // (head, entry) of the first page; every role then steps them incrementally
+    const int h_start = (int)(g0 / p.nwalk);
+    const int e_start = (int)(g0 - (long long)h_start * p.nwalk);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -364,15 +370,13 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         if (lane == 0) {
             int issued = 0;
             bool ok = true;
+            int h = h_start, e = e_start;
             for (int j = 0; j < J; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages && !wait_bar(kv_empty(st), ((j / kStages) - 1) & 1, ctl)) {
                     ok = false;
                     break;
                 }
-                const long long g = g0 + j;
-                const int h = (int)(g / p.nwalk);
-                const int e = (int)(g - (long long)h * p.nwalk);
                 const int page = __ldg(&p.walk[e].x);
                 if (page < 0 || page >= p.num_pages) {
                     *abort_flag = 1;
@@ -386,6 +390,10 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 tma_load_2d(dst, &tmK, 0, y, kv_full(st));
                 tma_load_2d(dst + L::kTileBytes, &tmV, 0, y, kv_full(st));
                 ++issued;
+                if (++e == p.nwalk) {
+                    e = 0;
+                    ++h;
+                }
             }
             if (!ok) {
                 // let every load already issued land before the CTA exits
@@ -400,49 +408,60 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_bf16(kRows, PAGE, false);
             constexpr uint32_t kIdescPV = idesc_bf16(kRows, 64, true);
-            auto qk = [&](int t, int j) {
-                const uint32_t kaddr = sbase + (j % kStages) * L::kStageBytes;
+            // descriptors of stage 0; stage s and step kk add constants to the
+            // start-address field (16-byte units): K steps 32 bytes, V steps 2 KB
+            const uint64_t kdesc0 = desc_sw128(sbase, 16, 1024);
+            const uint64_t vdesc0 = desc_sw128(sbase + L::kTileBytes, L::kTileBytes, 1024);
+            constexpr uint64_t kStageStep = L::kStageBytes >> 4;
+            auto qk = [&](int t, int st) {
+                const uint64_t kd = kdesc0 + st * kStageStep;
                 const uint32_t scol = tmem + L::kColS + t * PAGE;
+                const uint32_t qcol = tmem + L::kColQ + t * 32;
+                mma_ts(scol, qcol, kd, kIdescQK, 0u);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)   // 16 head dims per step
-                    mma_ts(scol, tmem + L::kColQ + t * 32 + kk * 8,
-                           desc_sw128(kaddr + kk * 32, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                for (int kk = 1; kk < 4; ++kk)   // 16 head dims per step
+                    mma_ts(scol, qcol + kk * 8, kd + 2 * kk, kIdescQK, 1u);
                 mma_commit(s_full(t));
             };
-            auto pv = [&](int t, int j) -> bool {
+            auto pv = [&](int t, int j, int st, bool first) -> bool {
                 if (!wait_bar(p_full(t), j & 1, ctl)) return false;
                 fence_after();
-                const int st = j % kStages;
-                const uint32_t vaddr = sbase + st * L::kStageBytes + L::kTileBytes;
-                const bool first = (j == 0) || ((g0 + j) % p.nwalk == 0);
+                const uint64_t vd = vdesc0 + st * kStageStep;
+                const uint32_t ocol = tmem + L::kColO + t * 64;
                 const uint32_t pcol = tmem + L::kColS + t * PAGE;
+                mma_ts(ocol, pcol, vd, kIdescPV, first ? 0u : 1u);
 #pragma unroll
-                for (int kk = 0; kk < PAGE / 16; ++kk)   // 16 keys per step
-                    mma_ts(tmem + L::kColO + t * 64, pcol + kk * 8,
-                           desc_sw128(vaddr + kk * 2048, L::kTileBytes, 1024), kIdescPV,
-                           (first && kk == 0) ? 0u : 1u);
+                for (int kk = 1; kk < PAGE / 16; ++kk)   // 16 keys per step
+                    mma_ts(ocol, pcol + kk * 8, vd + 128 * kk, kIdescPV, 1u);
                 mma_commit(pv_done(t));
                 if (t == 1) mma_commit(kv_empty(st));
                 return true;
             };
             bool ok = true;
             int sidx = 0;
+            int e = e_start;
+            bool prev_first = false;
+            int st = 0, prev_st = 0;
             for (int j = 0; j < J; ++j) {
-                const bool seg_first = (j == 0) || ((g0 + j) % p.nwalk == 0);
+                const bool seg_first = (j == 0) || (e == 0);
                 if (seg_first && !wait_bar(q_ready(0), sidx & 1, ctl)) { ok = false; break; }
-                if (!wait_bar(kv_full(j % kStages), (j / kStages) & 1, ctl)) { ok = false; break; }
+                if (!wait_bar(kv_full(st), (j / kStages) & 1, ctl)) { ok = false; break; }
                 fence_after();
-                qk(0, j);
-                if (j > 0 && !pv(1, j - 1)) { ok = false; break; }
+                qk(0, st);
+                if (j > 0 && !pv(1, j - 1, prev_st, prev_first)) { ok = false; break; }
                 if (seg_first) {
                     if (!wait_bar(q_ready(1), sidx & 1, ctl)) { ok = false; break; }
                     ++sidx;
                     fence_after();
                 }
-                qk(1, j);
-                if (!pv(0, j)) { ok = false; break; }
+                qk(1, st);
+                if (!pv(0, j, st, seg_first)) { ok = false; break; }
+                prev_first = seg_first;
+                prev_st = st;
+                st = (st + 1 == kStages) ? 0 : st + 1;
+                if (++e == p.nwalk) e = 0;
             }
-            if (ok) pv(1, J - 1);
+            if (ok) pv(1, J - 1, prev_st, prev_first);
             // drain: every MMA issued above completes before TMEM is released
             mma_commit(drain);
             wait_bar(drain, 0, ctl, false);
@@ -489,13 +508,15 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         auto all_ok = [&](bool ok) { return __all_sync(0xffffffffu, ok); };
 
         float m_run = -INFINITY, l_run = 0.f;
-        load_q((int)(g0 / p.nwalk));
+        load_q(h_start);
         // walk entries are read one page ahead, off the critical path
-        int4 ent_next = __ldg(&p.walk[(int)(g0 % p.nwalk)]);
+        int4 ent_next = __ldg(&p.walk[e_start]);
+        int h = h_start, e = e_start - 1;
         for (int j = 0; j < J; ++j) {
-            const long long g = g0 + j;
-            const int h = (int)(g / p.nwalk);
-            const int e = (int)(g - (long long)h * p.nwalk);
+            if (++e == p.nwalk) {
+                e = 0;
+                ++h;
+            }
             const bool seg_first = (j == 0) || (e == 0);
             const bool seg_last = (j == J - 1) || (e == p.nwalk - 1);
             if (seg_first) {
@@ -510,42 +531,86 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             if (!all_ok(wait_bar(s_full(t), j & 1, ctl))) break;
             fence_after();
             uint32_t r[PAGE];
+            auto load_s = [&]() {
 #pragma unroll
-            for (int c = 0; c < PAGE / 32; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
-            tmem_wait_ld();
-            if (nvis < PAGE) {
+                for (int c = 0; c < PAGE / 32; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
+                tmem_wait_ld();
+                if (nvis < PAGE) {
 #pragma unroll
-                for (int c = 0; c < PAGE; ++c) r[c] = (c < nvis) ? r[c] : 0xff800000u;
-            }
-            // row max: 16 independent three-input max chains, then a tree
-            float acc[16];
+                    for (int c = 0; c < PAGE; ++c) r[c] = (c < nvis) ? r[c] : 0xff800000u;
+                }
+            };
+            // r <- 2^(s * scale_log2 - msub) in place; returns the row sum
+            auto exps = [&](float msub) -> float {
+                const uint64_t sl2v = f2(sl2, sl2);
+                const uint64_t nmv = f2(-msub, -msub);
+                uint64_t rs2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(r[i]);
-#pragma unroll
-            for (int c = 16; c + 32 <= PAGE; c += 32)
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    acc[i] = fmax3(acc[i], __uint_as_float(r[c + i]), __uint_as_float(r[c + 16 + i]));
-            if constexpr ((PAGE - 16) % 32 != 0) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] = fmaxf(acc[i], __uint_as_float(r[PAGE - 16 + i]));
-            }
-            const float a0 = fmax3(acc[0], acc[1], acc[2]), a1 = fmax3(acc[3], acc[4], acc[5]);
-            const float a2 = fmax3(acc[6], acc[7], acc[8]), a3 = fmax3(acc[9], acc[10], acc[11]);
-            const float a4 = fmax3(acc[12], acc[13], acc[14]);
-            const float mx = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, acc[15]), -INFINITY);
+                for (int c = 0; c < PAGE; c += 2) {
+                    const uint64_t x = ffma2(f2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nmv);
+                    float x0, x1, p0, p1;
+                    unf2(x, x0, x1);
+                    if (((c >> 1) & 15) < kPolyPairs) {
+                        exp2_poly2(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    }
+                    rs2[(c >> 1) & 3] = fadd2(rs2[(c >> 1) & 3], f2(p0, p1));
+                    r[c] = __float_as_uint(p0);
+                    r[c + 1] = __float_as_uint(p1);
+                }
+                float s0, s1, s2, s3, s4, s5, s6, s7;
+                unf2(rs2[0], s0, s1);
+                unf2(rs2[1], s2, s3);
+                unf2(rs2[2], s4, s5);
+                unf2(rs2[3], s6, s7);
+                return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            };
+            load_s();
 
-            const float mt = mx * sl2;
+            // Fast path: exponentiate against the running max without looking
+            // for this page's max.  Values up to 2^64 are exact enough (relative
+            // precision does not depend on scale) and far from overflow; a row
+            // whose page sum reaches 2^64 (or inf / NaN) takes the exact path.
             float alpha = 1.f;
             bool resc = false;
-            if (mt > m_run + kRescaleThreshold) {
-                if (m_run != -INFINITY) {
-                    alpha = ex2(m_run - mt);
-                    resc = true;
-                }
-                m_run = mt;
+            bool fast = m_run != -INFINITY;
+            float rs = 0.f;
+            if (fast) {
+                rs = exps(m_run);
+                fast = rs < 0x1p64f;
             }
-            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+            if (!__all_sync(0xffffffffu, fast)) {
+                // r was overwritten by a fast attempt in some lanes; the reload is
+                // warp-collective, so every lane of the warp takes it
+                if (__any_sync(0xffffffffu, m_run != -INFINITY)) load_s();
+                // exact row max: 16 independent three-input max chains, then a tree
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(r[i]);
+#pragma unroll
+                for (int c = 16; c + 32 <= PAGE; c += 32)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        acc[i] = fmax3(acc[i], __uint_as_float(r[c + i]), __uint_as_float(r[c + 16 + i]));
+                if constexpr ((PAGE - 16) % 32 != 0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[i] = fmaxf(acc[i], __uint_as_float(r[PAGE - 16 + i]));
+                }
+                const float a0 = fmax3(acc[0], acc[1], acc[2]), a1 = fmax3(acc[3], acc[4], acc[5]);
+                const float a2 = fmax3(acc[6], acc[7], acc[8]), a3 = fmax3(acc[9], acc[10], acc[11]);
+                const float a4 = fmax3(acc[12], acc[13], acc[14]);
+                const float mt = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, acc[15]), -INFINITY) * sl2;
+                if (mt > m_run) {
+                    if (m_run != -INFINITY) {
+                        alpha = ex2(m_run - mt);
+                        resc = true;
+                    }
+                    m_run = mt;
+                }
+                rs = exps(m_run == -INFINITY ? 0.f : m_run);
+            }
 
             if (__any_sync(0xffffffffu, resc)) {
                 // PV_t(j-1) has completed (covered by the s_full commit)
@@ -566,37 +631,16 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 }
             }
 
-            // P = 2^(s * scale_log2 - m), packed bf16, written over the S columns
-            const uint64_t sl2v = f2(sl2, sl2);
-            const uint64_t nmv = f2(-msub, -msub);
-            uint64_t rs2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+            // P (bf16) written over the S columns
 #pragma unroll
             for (int c = 0; c < PAGE / 32; ++c) {
                 uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = ffma2(f2(__uint_as_float(r[32 * c + 2 * i]),
-                                                __uint_as_float(r[32 * c + 2 * i + 1])),
-                                             sl2v, nmv);
-                    float x0, x1, p0, p1;
-                    unf2(x, x0, x1);
-                    if (i < kPolyPairs) {
-                        exp2_poly2(x0, x1, p0, p1);
-                    } else {
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                    }
-                    rs2[i & 3] = fadd2(rs2[i & 3], f2(p0, p1));
-                    pk[i] = pack_bf16(p0, p1);
-                }
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16(__uint_as_float(r[32 * c + 2 * i]), __uint_as_float(r[32 * c + 2 * i + 1]));
                 tmem_st16(t_s + 16 * c, pk);
             }
-            float s0, s1, s2, s3, s4, s5, s6, s7;
-            unf2(rs2[0], s0, s1);
-            unf2(rs2[1], s2, s3);
-            unf2(rs2[2], s4, s5);
-            unf2(rs2[3], s6, s7);
-            l_run = l_run * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+            l_run = l_run * alpha + rs;
             tmem_wait_st();
             fence_before();
             mbar_arrive(p_full(t));
