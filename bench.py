@@ -54,6 +54,10 @@ def parse():
                     help="target CPU seconds of the oracle sample")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (profiling captures of a smaller case)")
+    ap.add_argument("--report", action="store_true",
+                    help="instead of the bench line: per-layer attention / append timings of "
+                         "the worked-example stream at T=100/1000/10000, the dense causal "
+                         "limit at T=1000 and one windowed-VO window, one JSON line each")
     return ap.parse_args()
 
 
@@ -197,9 +201,9 @@ class OracleSample:
 
 
 def calibrated_rows(sample, q0, last, seconds):
-    g, a = sample.run(q0, last, [0, 1])
-    per_row = a / 2
-    n = int(max(2, min(sample.w.Lq, seconds / max(per_row, 1e-6))))
+    g, a = sample.run(q0, last, list(range(16)))
+    per_row = a / 16
+    n = int(max(16, min(sample.w.Lq, seconds / max(per_row, 1e-6))))
     return list(range(n)), per_row
 
 
@@ -403,6 +407,77 @@ def run_ours(args, rank, world, local_rank):
     cache.close()
 
 
+def _time_ms(fn, reps=20, warm=3):
+    for _ in range(warm):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_report(args):
+    """Attention and append timings per layer on the other workloads."""
+    pk = peaks()
+    dev = torch.device("cuda", 0)
+
+    def emit(w, T, attend_ms, append_ms, note=""):
+        lk = lk_at(w, T)
+        fl = 4.0 * w.Lq * lk * w.H * w.D
+        print(json.dumps({"workload": w.name, "T": T, "Lq": w.Lq, "Lk": lk,
+                          "attend_ms": attend_ms, "append_ms_per_layer": append_ms,
+                          "tflops": fl / attend_ms / 1e9, "frac_bf16_peak": fl / attend_ms / 1e9 / pk["bf16"],
+                          "frames_per_s_per_layer": 1e3 / (attend_ms + append_ms), "note": note}),
+              flush=True)
+
+    def stream(w, T_points, max_frames):
+        cache = gca.Cache.for_workload(w, max_frames=max_frames)
+        out = torch.empty((1, w.Lq, w.H, w.D), dtype=torch.bfloat16, device=dev)
+        for t in range(max(T_points)):
+            k = inputs.draw(w, t, "k", dev)
+            v = inputs.draw(w, t, "v", dev)
+            if t + 1 in T_points:
+                q = inputs.draw(w, t, "q", dev)
+                # append time of this frame (one layer), then attention at T = t+1
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                cache.append(k, v)
+                e1.record()
+                cache.evict()
+                torch.cuda.synchronize()
+                app = e0.elapsed_time(e1)
+                att = _time_ms(lambda: cache.attend(0, q, out))
+                emit(w, t + 1, att, app)
+            else:
+                cache.append(k, v)
+                cache.evict()
+        cache.close()
+
+    stream(inputs.WORKED_EXAMPLE, {100, 1000, 10000}, 10000)
+    stream(inputs.DENSE_CAUSAL, {1000}, 1000)
+    vo = inputs.WINDOWED_VO
+    start, ln = vo.windows()[1]
+    cache = gca.Cache.for_workload(vo)
+    out = torch.empty((1, vo.Lq, vo.H, vo.D), dtype=torch.bfloat16, device=dev)
+    tot = 0.0
+    for t in range(ln):
+        k, v, q = (inputs.draw(vo, start + t, x, dev) for x in "kvq")
+        cache.append(k, v)
+        cache.evict()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        cache.attend(0, q, out)
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    print(json.dumps({"workload": vo.name, "window": [start, ln], "mean_attend_ms": tot / ln,
+                      "note": "mean over the 128 steps of window 1 after a reset"}), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -413,6 +488,9 @@ def main():
             run_reference(args)
         return
     torch.cuda.set_device(local_rank)
+    if args.report:
+        run_report(args)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

@@ -187,6 +187,14 @@ int gca_get_info(const gca_cache_t* cache, gca_info_t* info);
  * resets it. */
 int gca_device_status(gca_cache_t* cache, int32_t* status_out, int32_t clear);
 
+/* Failure-detection self-test: runs the kernels' bounded mbarrier wait on a
+ * barrier phase that nothing completes, with a deadline of timeout_ms (1 ..
+ * 10000).  The wait gives up, raises the cache's device status word and the
+ * kernel returns; the call synchronises the device and writes the status word
+ * (1 = a wait ran out) to *status_out.  Clear it with gca_device_status(.., 1)
+ * before further calls on the cache. */
+int gca_selftest_bounded_wait(gca_cache_t* cache, int32_t timeout_ms, int32_t* status_out);
+
 /* Static text of a status code. */
 const char* gca_status_string(int status);
 

@@ -360,3 +360,25 @@ def test_dense_causal_limit_T1000():
     res = _stream(w, cache, sim, mirror, w.T, {999}, [0], rows)
     assert cache.info().resident_tokens == 1005 * 1000
     print("dense limit errors", res)
+
+
+def test_bounded_wait_reports_instead_of_hanging():
+    """A kernel wait that can never complete gives up after its deadline,
+    raises the status word, and leaves the context usable: the next calls
+    run and still match the oracle."""
+    w = inputs.TINY_BF16
+    cache = gca.Cache.for_workload(w)
+    assert gca.gca_selftest_bounded_wait(cache.handle, 100) == 1
+    k, v, q = (inputs.draw(w, 0, x).cuda() for x in "kvq")
+    with pytest.raises(gca.GCAError) as e:
+        cache.append(k, v)                      # the raised status word is reported
+    assert e.value.name == "GCA_ERR_DEVICE_CHECK"
+    assert cache.status(clear=True) == 1
+    mirror = Mirror(w, [0])
+    cache.append(k, v)
+    mirror.record(0, k, v, keep_full=True)
+    out, _ = attend(cache, 0, q)
+    want, _ = oracle_step(mirror, 0, q.float().cpu().numpy(), 0)
+    torch.cuda.synchronize()
+    assert max_err(out, want) <= TOL["bf16"]
+    assert cache.status() == 0

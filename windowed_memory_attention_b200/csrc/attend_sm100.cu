@@ -133,14 +133,15 @@ struct Ctl {
 };
 
 // Bounded parity wait.  honour_abort = false is used while draining.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, bool honour_abort = true) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, bool honour_abort = true,
+                                         unsigned long long timeout_ns = kTimeoutNs) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(bar, parity)) return true;
         if ((it & 127u) == 0) {
             if (honour_abort && *c.abort) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
+            if (globaltimer() - t0 > timeout_ns) {
                 *c.abort = 1;
                 *(volatile int*)c.status = kStatusWaitTimeout;
                 __threadfence_system();
@@ -696,6 +697,20 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     }
 }
 
+// Self-test of the bounded wait: one thread waits on a barrier phase that
+// nothing completes; the wait gives up after timeout_ns, raises the status
+// word and the kernel returns.
+__global__ void bounded_wait_selftest(int* status, unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const Ctl ctl{&abort_flag, status};
+    wait_bar(smem_u32(&bar), 0, ctl, true, timeout_ns);
+}
+
 // Combine the partials of heads that were split between workers.
 __global__ void __launch_bounds__(128) merge_kernel(const AttendParams p) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -761,6 +776,11 @@ cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
     if (p.P == 128) return launch_page<128>(tk, tv, p, s);
     if (p.P == 64) return launch_page<64>(tk, tv, p, s);
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bounded_wait_selftest(int* status, unsigned long long timeout_ns, cudaStream_t s) {
+    bounded_wait_selftest<<<1, 32, 0, s>>>(status, timeout_ns);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_merge(const AttendParams& p, cudaStream_t s) {

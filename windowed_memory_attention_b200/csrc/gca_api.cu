@@ -464,6 +464,18 @@ int gca_device_status(gca_cache_t* c, int32_t* status_out, int32_t clear) {
     return GCA_OK;
 }
 
+int gca_selftest_bounded_wait(gca_cache_t* c, int32_t timeout_ms, int32_t* status_out) {
+    if (!c || !status_out || timeout_ms < 1 || timeout_ms > 10000) return GCA_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    if (gca::launch_bounded_wait_selftest(c->d_status, (unsigned long long)timeout_ms * 1000000ull, 0) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return GCA_ERR_CUDA;
+    }
+    *status_out = *(volatile int*)c->h_status;
+    return GCA_OK;
+}
+
 int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* out, float* lse,
                void* stream) {
     if (!c || !q || !out) return GCA_ERR_INVALID_ARG;

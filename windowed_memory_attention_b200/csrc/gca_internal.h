@@ -79,6 +79,7 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
                                 const AttendParams& p, cudaStream_t s);
 cudaError_t launch_merge(const AttendParams& p, cudaStream_t s);
+cudaError_t launch_bounded_wait_selftest(int* status, unsigned long long timeout_ns, cudaStream_t s);
 cudaError_t launch_attend_f32(const AttendParams& p, const void* kpool, const void* vpool,
                               cudaStream_t s);
 

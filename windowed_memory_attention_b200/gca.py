@@ -24,7 +24,8 @@ STATUS = {0: "GCA_OK", 1: "GCA_ERR_INVALID_ARG", 2: "GCA_ERR_CAPACITY", 3: "GCA_
           4: "GCA_ERR_UNSUPPORTED", 5: "GCA_ERR_CUDA", 6: "GCA_ERR_DEVICE_CHECK"}
 EXPORTS = ("gca_cache_create", "gca_cache_destroy", "gca_append_frame", "gca_evict_to_summary",
            "gca_attend", "gca_reset", "gca_get_layout", "gca_token_slot", "gca_get_info",
-           "gca_device_status", "gca_status_string", "gca_attend_pages_noalloc")
+           "gca_device_status", "gca_status_string", "gca_attend_pages_noalloc",
+           "gca_selftest_bounded_wait")
 
 
 class gca_config_t(ctypes.Structure):
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "gca_token_slot": [vp, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
             "gca_get_info": [vp, ctypes.POINTER(gca_info_t)],
             "gca_device_status": [vp, ctypes.POINTER(i32), i32],
+            "gca_selftest_bounded_wait": [vp, i32, ctypes.POINTER(i32)],
             "gca_attend_pages_noalloc": [vp, vp, i32, i32, i32, i32, i32, vp, i32, vp, i32, i32,
                                          i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp],
         }
@@ -197,6 +199,12 @@ def gca_attend_pages_noalloc(k_pool, v_pool, *, num_layers: int, num_pages: int,
         _ptr(q), num_query_frames, tokens_per_frame, first_query_frame, num_anchor, window,
         summary_tokens, int(bool(anchor_block)), softmax_scale, _ptr(out), _ptr(lse),
         _ptr(status), _stream(stream)))
+
+
+def gca_selftest_bounded_wait(cache, timeout_ms: int = 100) -> int:
+    s = ctypes.c_int32(0)
+    _check("gca_selftest_bounded_wait", lib().gca_selftest_bounded_wait(cache, timeout_ms, ctypes.byref(s)))
+    return s.value
 
 
 class Cache:
