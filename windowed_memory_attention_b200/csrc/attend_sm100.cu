@@ -192,6 +192,15 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
         "r"(a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] += A[tmem] * B[smem desc]; B given as its two 32-bit halves
+__device__ __forceinline__ void mma_ts_acc(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc) {
+    asm volatile(
+        "{\n.reg .b64 bd;\nmov.b64 bd, {%2, %3};\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, 1;\n}" ::"r"(d),
+        "r"(a), "r"(b_lo), "r"(b_hi), "r"(idesc)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -414,55 +423,64 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             const uint64_t kdesc0 = desc_sw128(sbase, 16, 1024);
             const uint64_t vdesc0 = desc_sw128(sbase + L::kTileBytes, L::kTileBytes, 1024);
             constexpr uint64_t kStageStep = L::kStageBytes >> 4;
+            // descriptor halves: only the low word (start address) varies
+            const uint32_t kd_lo0 = (uint32_t)kdesc0, kd_hi = (uint32_t)(kdesc0 >> 32);
+            const uint32_t vd_lo0 = (uint32_t)vdesc0, vd_hi = (uint32_t)(vdesc0 >> 32);
             auto qk = [&](int t, int st) {
                 const uint64_t kd = kdesc0 + st * kStageStep;
+                const uint32_t kd_lo = kd_lo0 + st * (uint32_t)kStageStep;
                 const uint32_t scol = tmem + L::kColS + t * PAGE;
                 const uint32_t qcol = tmem + L::kColQ + t * 32;
                 mma_ts(scol, qcol, kd, kIdescQK, 0u);
 #pragma unroll
                 for (int kk = 1; kk < 4; ++kk)   // 16 head dims per step
-                    mma_ts(scol, qcol + kk * 8, kd + 2 * kk, kIdescQK, 1u);
+                    mma_ts_acc(scol, qcol + kk * 8, kd_lo + 2 * kk, kd_hi, kIdescQK);
                 mma_commit(s_full(t));
             };
-            auto pv = [&](int t, int j, int st, bool first) -> bool {
+            // pv_done is only needed at the end of a head: the commit after the
+            // next QK_t covers PV_t for the softmax
+            auto pv = [&](int t, int j, int st, bool first, bool last) -> bool {
                 if (!wait_bar(p_full(t), j & 1, ctl)) return false;
                 fence_after();
                 const uint64_t vd = vdesc0 + st * kStageStep;
+                const uint32_t vd_lo = vd_lo0 + st * (uint32_t)kStageStep;
                 const uint32_t ocol = tmem + L::kColO + t * 64;
                 const uint32_t pcol = tmem + L::kColS + t * PAGE;
                 mma_ts(ocol, pcol, vd, kIdescPV, first ? 0u : 1u);
 #pragma unroll
                 for (int kk = 1; kk < PAGE / 16; ++kk)   // 16 keys per step
-                    mma_ts(ocol, pcol + kk * 8, vd + 128 * kk, kIdescPV, 1u);
-                mma_commit(pv_done(t));
+                    mma_ts_acc(ocol, pcol + kk * 8, vd_lo + 128 * kk, vd_hi, kIdescPV);
+                if (last) mma_commit(pv_done(t));
                 if (t == 1) mma_commit(kv_empty(st));
                 return true;
             };
             bool ok = true;
             int sidx = 0;
             int e = e_start;
-            bool prev_first = false;
+            bool prev_first = false, prev_last = false;
             int st = 0, prev_st = 0;
             for (int j = 0; j < J; ++j) {
                 const bool seg_first = (j == 0) || (e == 0);
+                const bool seg_last = (j == J - 1) || (e == p.nwalk - 1);
                 if (seg_first && !wait_bar(q_ready(0), sidx & 1, ctl)) { ok = false; break; }
                 if (!wait_bar(kv_full(st), (j / kStages) & 1, ctl)) { ok = false; break; }
                 fence_after();
                 qk(0, st);
-                if (j > 0 && !pv(1, j - 1, prev_st, prev_first)) { ok = false; break; }
+                if (j > 0 && !pv(1, j - 1, prev_st, prev_first, prev_last)) { ok = false; break; }
                 if (seg_first) {
                     if (!wait_bar(q_ready(1), sidx & 1, ctl)) { ok = false; break; }
                     ++sidx;
                     fence_after();
                 }
                 qk(1, st);
-                if (!pv(0, j, st, seg_first)) { ok = false; break; }
+                if (!pv(0, j, st, seg_first, seg_last)) { ok = false; break; }
                 prev_first = seg_first;
+                prev_last = seg_last;
                 prev_st = st;
                 st = (st + 1 == kStages) ? 0 : st + 1;
                 if (++e == p.nwalk) e = 0;
             }
-            if (ok) pv(1, J - 1, prev_st, prev_first);
+            if (ok) pv(1, J - 1, prev_st, prev_first, prev_last);
             // drain: every MMA issued above completes before TMEM is released
             mma_commit(drain);
             wait_bar(drain, 0, ctl, false);
@@ -509,6 +527,7 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         auto all_ok = [&](bool ok) { return __all_sync(0xffffffffu, ok); };
 
         float m_run = -INFINITY, l_run = 0.f;
+        int segs_done = 0;                             // pv_done(t) phases consumed
         load_q(h_start);
         // walk entries are read one page ahead, off the critical path
         int4 ent_next = __ldg(&p.walk[e_start]);
@@ -647,7 +666,8 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             mbar_arrive(p_full(t));
 
             if (seg_last) {
-                if (!all_ok(wait_bar(pv_done(t), j & 1, ctl))) break;
+                if (!all_ok(wait_bar(pv_done(t), segs_done & 1, ctl))) break;
+                ++segs_done;
                 fence_after();
                 uint32_t o[64];
                 tmem_ld32(t_o, o);
