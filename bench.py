@@ -362,6 +362,28 @@ def run_ours(args, rank, world, local_rank):
 
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
+    # ---- non-keyframe step (untimed above): the frame reads the cache and its
+    # own tokens through gca_attend_transient and nothing is kept
+    qn, kn, vn = (inputs.draw(w, T_end + E + 7, x, dev) for x in "qkv")
+    outn = torch.empty((w.Lq, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    for l in range(w.L):
+        cache.attend_transient(l, qn[l], kn[l], vn[l], outn)
+    torch.cuda.synchronize(dev)
+    nk_ev = [(ev(), ev()) for _ in range(w.L)]
+    for l in range(w.L):
+        nk_ev[l][0].record(stream)
+        cache.attend_transient(l, qn[l], kn[l], vn[l], outn)
+        nk_ev[l][1].record(stream)
+    torch.cuda.synchronize(dev)
+    nk_ms = statistics.mean(a.elapsed_time(b) for (a, b) in nk_ev)
+    nk_keys = lk_at(w, cache.info().frames) + w.Lq
+    nonkey = {"ms_per_layer": nk_ms, "frames_per_s_per_layer": 1e3 / nk_ms, "keys": nk_keys,
+              "tflops": 4.0 * w.Lq * nk_keys * w.H * w.D / nk_ms / 1e9,
+              "note": "gca_attend_transient per layer: the frame's K/V into transient pages, then "
+                      "attention over the cache and the frame; page table unchanged"}
+    if cache.status() != 0:
+        raise RuntimeError(f"device status word raised: {cache.status()}")
+
     if rank != 0:
         return
     pk = peaks()
@@ -387,6 +409,7 @@ def run_ours(args, rank, world, local_rank):
         "append_roofline": {"bound": "hbm", "achieved": app_gbs, "peak": pk["hbm"],
                             "unit": "GB/s", "frac": app_gbs / pk["hbm"],
                             "bytes_per_launch": app_bytes, "avg_launch_ms": statistics.mean(app_ms)},
+        "nonkey_step": nonkey,
         "gpu_launches": int(launches),
         "clocks": clk,
         "e2e": e2e,
@@ -452,6 +475,15 @@ def run_report(args):
                 app = e0.elapsed_time(e1)
                 att = _time_ms(lambda: cache.attend(0, q, out))
                 emit(w, t + 1, att, app)
+                # a non-keyframe at the same state: reads the cache and its own tokens
+                qn, kn, vn = (inputs.draw(w, 10 ** 6 + t, x, dev)[0] for x in "qkv")
+                outn = torch.empty((w.Lq, w.H, w.D), dtype=torch.bfloat16, device=dev)
+                att_n = _time_ms(lambda: cache.attend_transient(0, qn, kn, vn, outn))
+                lk = lk_at(w, t + 1) + w.Lq
+                fl = 4.0 * w.Lq * lk * w.H * w.D
+                print(json.dumps({"workload": w.name, "T": t + 1, "step": "non-keyframe",
+                                  "Lk": lk, "ms_per_layer": att_n, "tflops": fl / att_n / 1e9,
+                                  "frames_per_s_per_layer": 1e3 / att_n}), flush=True)
             else:
                 cache.append(k, v)
                 cache.evict()

@@ -118,9 +118,12 @@ typedef struct {
 
 /* Create a cache on CUDA device `device`.  Allocates both pools:
  * num_pages = (n + k + max_query_frames + frame_slack) * ceil(M/P)
- *           + ceil(S * max_frames / P)  pages per layer.
+ *           + ceil(S * max_frames / P)   pages the allocator hands out,
+ *           + ceil((S+M) / P)            transient pages after them
+ *                                        (gca_attend_transient), per layer.
  * Errors: INVALID_ARG (non-positive sizes, null out), UNSUPPORTED (head_dim
- * != 64, page_size not 64/128, unknown dtype), CUDA (allocation). */
+ * != 64, page_size not 64/128, unknown dtype, ceil((S+M)/P) > 128), CUDA
+ * (allocation). */
 int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out);
 
 /* Free everything the cache owns.  The caller must have synchronised the
@@ -161,6 +164,25 @@ int gca_evict_to_summary(gca_cache_t* cache, int32_t* frames_evicted_out);
  * INVALID_ARG (F < 1 or F > max_query_frames), DEVICE_CHECK. */
 int gca_attend(gca_cache_t* cache, int32_t layer, const void* q, int32_t num_query_frames,
                void* out, float* lse, void* stream);
+
+/* Non-keyframe step for one layer (code walkthrough §3.2, keyframe_interval;
+ * paper digest §5.1, keyframe selection): a frame that is not a keyframe is
+ * predicted like any other, but its K and V never enter the cache.  Its
+ * queries attend to every token the cache holds for `layer` — what the latest
+ * keyframe t = T-1 reads as a single query frame (anchors, its window, every
+ * summary token) — and to the frame's own S+M tokens (bidirectional), with
+ * softmax(scale * q.k) and fp32 accumulation.  With no keyframe yet (T = 0) it
+ * reads only its own tokens.
+ * q, k, v: [S+M][H][D] of this layer (summary tokens first), device or host
+ * memory; out [S+M][H][D] in the cache dtype; lse (nullable) [S+M][H]
+ * float32, natural log.  k and v are copied into ceil((S+M)/P) transient pages
+ * of this layer (past the allocator's pages) and are dropped by the next call
+ * for the layer: the page table, frame count and eviction state do not
+ * change, so calls for one layer must be ordered (one stream).
+ * Errors: STATE (layer has not appended frame T-1, or a frame the latest
+ * keyframe needs was evicted), INVALID_ARG, DEVICE_CHECK. */
+int gca_attend_transient(gca_cache_t* cache, int32_t layer, const void* q, const void* k,
+                         const void* v, void* out, float* lse, void* stream);
 
 /* Back to the creation state (windowed mode: state is reset at each window
  * start; code walkthrough §3.3).  Page tables become identical to a fresh

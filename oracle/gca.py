@@ -22,7 +22,10 @@ Sources (LingBot-Map pages):
   * news article, mask figure caption (d): GCA with n=2 anchors, k=2 window;
   * code walkthrough §2: a frame that leaves the window drops its M image tokens
     and keeps its summary tokens; §3.2: anchors ("scale frames") form one block
-    that attends within itself before single-frame streaming.
+    that attends within itself before single-frame streaming, and with
+    keyframe_interval > 1 a non-keyframe is predicted from the cache but its
+    K/V is not kept (skip-append); §3.3: the window counts keyframes entering
+    the cache, not video frames.
 
 Readings where the pages leave a step open (each is listed in the design doc):
   * the k-frame window counts the current frame, so after frame t the full
@@ -30,7 +33,9 @@ Readings where the pages leave a step open (each is listed in the design doc):
     cache holds exactly M(n+k)+6T tokens once T > n+k;
   * attention inside a frame is bidirectional; causality is per frame;
   * the summary tokens of anchor and window frames are counted once;
-  * in the anchor-block option the n anchors see each other's tokens in full.
+  * in the anchor-block option the n anchors see each other's tokens in full;
+  * a non-keyframe reads exactly what the latest keyframe reads as a single
+    query frame, plus all of its own tokens (bidirectional).
 
 Parity pins: tests/test_oracle_pins.py.  The one unpinned quantity is the
 model's learned numbers, which this path does not compute.
@@ -222,6 +227,78 @@ def stream_step(q_block: np.ndarray, last_frame: int, frame_kv: FrameKV, *, n: i
         kk, vv = gather_keys(i, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block)
         qi = q_block[b] if rows is None else q_block[b][list(rows)]
         o, l = attention(qi, kk, vv, scale, impl)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+# ----------------------------------------------------------------------------
+# non-keyframe steps (code walkthrough §3.2: keyframe_interval; paper digest
+# §5.1: not every frame enters the memory)
+# ----------------------------------------------------------------------------
+def is_keyframe(x: int, *, n: int, interval: int) -> bool:
+    """Does video frame x enter the cache?  The first n (scale) frames always
+    do; after them every interval-th frame, counting from frame n, does."""
+    return x < n or interval <= 1 or (x - n) % interval == 0
+
+
+def latest_keyframe(x: int, *, n: int, interval: int) -> int:
+    """Cache index of the latest keyframe among video frames 0..x (the cache
+    numbers keyframes 0, 1, 2, ... in the order they enter); -1 if none."""
+    return sum(1 for y in range(x + 1) if is_keyframe(y, n=n, interval=interval)) - 1
+
+
+def transient_step(q: np.ndarray, own_k: np.ndarray, own_v: np.ndarray, last_key: int,
+                   frame_kv: FrameKV, *, n: int, k: int, S: int, scale: float,
+                   anchor_block: bool = False, rows: Optional[Sequence[int]] = None,
+                   impl: str = "c"):
+    """Output of a non-keyframe, q / own_k / own_v [S+M][H][D].
+
+    The frame is predicted like every other frame but its K/V never enters the
+    cache: its queries read what the latest keyframe (cache index last_key)
+    reads as a single query frame, plus all of its own tokens.  With no
+    keyframe yet (last_key < 0) they read only their own tokens.  Returns out
+    [R][H][D] and lse [R][H] in float64.
+    """
+    ks, vs = [], []
+    if last_key >= 0:
+        kk, vv = gather_keys(last_key, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block)
+        ks.append(kk)
+        vs.append(vv)
+    ks.append(own_k)
+    vs.append(own_v)
+    qi = q if rows is None else q[list(rows)]
+    return attention(qi, np.concatenate(ks, 0), np.concatenate(vs, 0), scale, impl)
+
+
+def bruteforce_keyframes(Q: np.ndarray, K: np.ndarray, V: np.ndarray, *, n: int, k: int,
+                         S: int, interval: int, scale: float, anchor_block: bool = False):
+    """Every video frame's output at once for a stream in which only keyframes
+    are cached.  Q, K, V [X][S+M][H][D] over all X video frames.  A query of
+    frame x sees token tau of keyframe y when the token rule allows it between
+    the cache indices of x's latest keyframe and of y, and, when x itself is
+    not a keyframe, every token of x.  Returns out [X][S+M][H][D], lse
+    [X][S+M][H] (float64)."""
+    X, Lq, H, D = Q.shape
+    kid = {}
+    for y in range(X):
+        if is_keyframe(y, n=n, interval=interval):
+            kid[y] = len(kid)
+    q = Q.astype(np.float64)
+    kf = K.reshape(X * Lq, H, D).astype(np.float64)
+    vf = V.reshape(X * Lq, H, D).astype(np.float64)
+    outs, lses = [], []
+    for x in range(X):
+        i = latest_keyframe(x, n=n, interval=interval)
+        vis = np.zeros(X * Lq, dtype=bool)
+        for y in range(X):
+            for tau in range(Lq):
+                if y in kid and i >= 0:
+                    vis[y * Lq + tau] = visible(i, kid[y], tau, n=n, k=k, S=S,
+                                                anchor_block=anchor_block)
+                if y == x and x not in kid:
+                    vis[y * Lq + tau] = True
+        o, l = attention_np(q[x], kf[vis], vf[vis], scale)
         outs.append(o)
         lses.append(l)
     return np.stack(outs), np.stack(lses)

@@ -69,6 +69,26 @@ def oracle_step(mirror: Mirror, layer: int, q_block: np.ndarray, last: int, F: i
                             scale=w.softmax_scale, anchor_block=anchor_block, rows=rows)
 
 
+def oracle_transient(mirror: Mirror, layer: int, q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                     last_key: int, rows=None, anchor_block: bool = False):
+    """Oracle output of a non-keyframe (q, k, v [S+M][H][D], all heads) that
+    reads the cache after keyframe last_key plus its own tokens."""
+    w = mirror.w
+    if mirror.heads is not None:
+        q, k, v = q[:, mirror.heads], k[:, mirror.heads], v[:, mirror.heads]
+    return ogca.transient_step(q, k, v, last_key, mirror.frame_kv(layer), n=w.n, k=w.k, S=w.S,
+                               scale=w.softmax_scale, anchor_block=anchor_block, rows=rows)
+
+
+def attend_transient(cache: gca.Cache, layer: int, q: torch.Tensor, k: torch.Tensor,
+                     v: torch.Tensor):
+    """q, k, v: [S+M][H][D] on the GPU; returns (out, lse) on the GPU."""
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    cache.attend_transient(layer, q, k, v, out, lse)
+    return out, lse
+
+
 def attend(cache: gca.Cache, layer: int, q: torch.Tensor, F: int = 1):
     """q: [F][S+M][H][D] on the GPU; returns (out, lse) on the GPU."""
     out = torch.empty_like(q)

@@ -13,7 +13,8 @@ import torch
 
 from oracle.allocator import PageTableSim
 from windowed_memory_attention_b200 import gca, inputs
-from gca_stream_util import Mirror, attend, max_err, needed_full, oracle_step, pool_view
+from gca_stream_util import (Mirror, attend, attend_transient, max_err, needed_full, oracle_step,
+                             oracle_transient, pool_view)
 
 pytestmark = pytest.mark.gpu
 
@@ -265,11 +266,79 @@ def test_page_size_64():
 
 
 # ----------------------------------------------------------------------------
+# non-keyframe steps: only keyframes enter the cache
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("interval", [2, 3])
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
+def test_keyframe_interval_stream(w, interval):
+    """Video frames 0..T-1; keyframes (the n scale frames, then every
+    interval-th frame) are appended and evicted, the others attend through
+    gca_attend_transient and leave the page table untouched."""
+    cache = gca.Cache.for_workload(w)
+    sim = _sim(w)
+    mirror = Mirror(w, range(w.L))
+    kid = -1
+    n_trans = 0
+    for x in range(w.T):
+        k = inputs.draw(w, x, "k").cuda()
+        v = inputs.draw(w, x, "v").cuda()
+        q = inputs.draw(w, x, "q").cuda()
+        if x < w.n or (x - w.n) % interval == 0:
+            kid += 1
+            assert cache.append(k, v) == kid
+            sim.append()
+            mirror.record(kid, k, v, keep_full=True)
+            assert cache.evict() == sim.evict()
+            out, _ = attend(cache, 0, q[0:1].contiguous())
+            want, _ = oracle_step(mirror, 0, q[0:1].float().cpu().numpy(), kid)
+            torch.cuda.synchronize()
+            assert max_err(out[0], want[0]) <= TOL[w.dtype], x
+            continue
+        launches = cache.info().kernel_launches
+        for l in range(w.L):
+            out, lse = attend_transient(cache, l, q[l], k[l], v[l])
+            want, wlse = oracle_transient(mirror, l, q[l].float().cpu().numpy(),
+                                          k[l].float().cpu().numpy(), v[l].float().cpu().numpy(), kid)
+            torch.cuda.synchronize()
+            assert max_err(out, want) <= TOL[w.dtype], (x, l)
+            assert max_err(lse, wlse) <= LSE_TOL[w.dtype], (x, l)
+        n_trans += 1
+        # nothing was kept: same frame count, tables and resident tokens
+        assert cache.layout() == sim.walk()
+        info = cache.info()
+        assert info.frames == kid + 1 and info.resident_tokens == sim.resident_tokens()
+        assert info.kernel_launches > launches
+    assert n_trans > 0 and cache.status() == 0
+
+
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
+def test_transient_before_any_keyframe_and_host_pointers(w):
+    """With an empty cache a non-keyframe reads only its own tokens; host
+    tensors give the same result as device tensors."""
+    cache = gca.Cache.for_workload(w)
+    mirror = Mirror(w, [0])
+    q, k, v = (inputs.draw(w, 5, x)[0] for x in "qkv")
+    out, lse = attend_transient(cache, 0, q.cuda(), k.cuda(), v.cuda())
+    want, wlse = oracle_transient(mirror, 0, q.float().numpy(), k.float().numpy(), v.float().numpy(), -1)
+    torch.cuda.synchronize()
+    assert max_err(out, want) <= TOL[w.dtype]
+    assert max_err(lse, wlse) <= LSE_TOL[w.dtype]
+    out_h = torch.empty_like(q).pin_memory()
+    lse_h = torch.empty(q.shape[:2], dtype=torch.float32).pin_memory()
+    cache.attend_transient(0, q.pin_memory(), k.pin_memory(), v.pin_memory(), out_h, lse_h)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, out.cpu()) and torch.equal(lse_h, lse.cpu())
+    assert cache.info().frames == 0
+
+
+# ----------------------------------------------------------------------------
 # the larger workloads
 # ----------------------------------------------------------------------------
-def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, reset=False):
+def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, reset=False,
+            transient=False):
     """Stream frames frame0..frame0+T-1 (local indices 0..T-1); at each local
-    step in `checks` compare sampled rows of the listed layers with the oracle."""
+    step in `checks` compare sampled rows of the listed layers with the oracle
+    (and, with `transient`, a non-keyframe's attention at that state)."""
     dev = "cuda"
     if reset:
         cache.reset()
@@ -301,6 +370,21 @@ def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, r
                 assert e <= TOL["bf16"], (t, l, e)
                 assert el <= LSE_TOL["bf16"], (t, l, el)
                 assert torch.isfinite(out).all()
+                if transient:
+                    # a non-keyframe (tensors of a frame outside the stream)
+                    qt, kt, vt = (inputs.draw(w, frame0 + T + 1, x, dev, layers=[l])[0] for x in "qkv")
+                    out, lse = attend_transient(cache, l, qt, kt, vt)
+                    torch.cuda.synchronize()
+                    want, wlse = oracle_transient(mirror, l, qt.float().cpu().numpy(), kt.float().cpu().numpy(),
+                                                  vt.float().cpu().numpy(), t, rows=rows)
+                    got, gl = out[rows], lse[rows]
+                    if heads is not None:
+                        got, gl = got[:, heads], gl[:, heads]
+                    e = max_err(got, want)
+                    results.append((t, l, "transient", e))
+                    assert e <= TOL["bf16"], (t, l, "transient", e)
+                    assert max_err(gl, wlse) <= LSE_TOL["bf16"], (t, l, "transient")
+                    assert cache.layout() == sim.walk()
             mirror.drop_full(set(f for f in range(t + 1) if f < w.n) |
                              set(f for c in checks if c > t for f in range(max(0, c - w.k + 1), t + 1)))
     assert cache.status() == 0
@@ -313,7 +397,7 @@ def test_worked_example_to_T10000():
     sim = _sim(w)
     mirror = Mirror(w, [0])
     rows = _rows_sample(w.Lq, extra=12)
-    res = _stream(w, cache, sim, mirror, w.T, {99, 999, 9999}, [0], rows)
+    res = _stream(w, cache, sim, mirror, w.T, {99, 999, 9999}, [0], rows, transient=True)
     assert cache.info().resident_tokens == 500 * 19 + 6 * 10000
     print("worked example max errors", res)
 
@@ -324,7 +408,7 @@ def test_metric_workload_T10000_all_layers():
     sim = _sim(w)
     mirror = Mirror(w, [0, 23])
     rows = _rows_sample(w.Lq, extra=8, seed=3)
-    res = _stream(w, cache, sim, mirror, w.T, {9999}, [0, 23], rows)
+    res = _stream(w, cache, sim, mirror, w.T, {9999}, [0, 23], rows, transient=True)
     assert cache.info().resident_tokens == 999 * 67 + 6 * 10000
     # every layer's output at T=10000 is finite and its lse lies within the
     # bounds softmax attention allows: ln(#keys) - max|s| <= lse <= ln(#keys) + max|s|

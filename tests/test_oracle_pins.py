@@ -112,6 +112,70 @@ def pin_causal_limit_sdpa(M=7, n=2, k=6, T=6, H=2, D=16, seed=3):
     return bool(np.abs(o1 - ref).max() < 1e-12 and np.abs(o2 - ref).max() < 1e-12)
 
 
+def _o1_keyframes(Q, K, V, *, n, k, S, interval, scale, impl="np"):
+    """O1 over a stream in which only keyframes are cached: keyframes through
+    stream_step on the keyframe sequence, the others through transient_step."""
+    keys = [y for y in range(Q.shape[0]) if gca.is_keyframe(y, n=n, interval=interval)]
+    fkv = _frame_kv(K[keys], V[keys])
+    outs, lses = [], []
+    for x in range(Q.shape[0]):
+        i = gca.latest_keyframe(x, n=n, interval=interval)
+        if gca.is_keyframe(x, n=n, interval=interval):
+            o, l = gca.stream_step(Q[x:x + 1], i, fkv, n=n, k=k, S=S, scale=scale, impl=impl)
+            o, l = o[0], l[0]
+        else:
+            o, l = gca.transient_step(Q[x], K[x], V[x], i, fkv, n=n, k=k, S=S, scale=scale,
+                                      impl=impl)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+def pin_transient_before_eviction_is_sdpa(M=5, n=2, k=8, X=9, interval=2, H=2, D=16, seed=21):
+    """While nothing has been evicted a non-keyframe sees every token of the
+    cached keyframes and of itself: plain attention (torch SDPA, fp64)."""
+    Q, K, V = _rand_stream(X, M, H, D, seed)
+    scale = 1 / math.sqrt(D)
+    keys = [y for y in range(X) if gca.is_keyframe(y, n=n, interval=interval)]
+    assert len(keys) <= n + k                      # no eviction in this stream
+    fkv = _frame_kv(K[keys], V[keys])
+    checked = 0
+    for x in range(X):
+        if gca.is_keyframe(x, n=n, interval=interval):
+            continue
+        i = gca.latest_keyframe(x, n=n, interval=interval)
+        o, _ = gca.transient_step(Q[x], K[x], V[x], i, fkv, n=n, k=k, S=6, scale=scale, impl="np")
+        seen = keys[:i + 1] + [x]
+        kk = torch.from_numpy(K[seen].astype(np.float64)).reshape(-1, H, D).permute(1, 0, 2)
+        vv = torch.from_numpy(V[seen].astype(np.float64)).reshape(-1, H, D).permute(1, 0, 2)
+        qq = torch.from_numpy(Q[x].astype(np.float64)).permute(1, 0, 2)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)
+        if np.abs(o - ref.permute(1, 0, 2).numpy()).max() > 1e-12:
+            return False
+        checked += 1
+    return checked > 0
+
+
+def pin_transient_key_count(M=5, S=6, n=2, k=3, X=17, interval=3, H=1, D=8):
+    """Q = 0: lse = ln(#keys read) = ln(cache size after the latest keyframe
+    (closed form) + the frame's own S+M tokens)."""
+    Q, K, V = _rand_stream(X, M, H, D, seed=9, S=S)
+    Q[:] = 0
+    try:
+        _, lse = _o1_keyframes(Q, K, V, n=n, k=k, S=S, interval=interval, scale=0.125)
+    except (ValueError, IndexError):
+        return False                  # an oracle that cannot even run fails the pin
+    for x in range(X):
+        # keyframes among video frames 0..x, counted directly: all of the first
+        # n, then frames n, n+interval, n+2*interval, ...
+        cached = x + 1 if x < n else n + (x - n) // interval + 1
+        own = 0 if (x < n or (x - n) % interval == 0) else S + M
+        want = math.log(gca.cache_tokens(M, S, n, k, cached) + own)
+        if not np.allclose(lse[x], want, atol=1e-12, rtol=0):
+            return False
+    return True
+
+
 # ----------------------------------------------------------------------------
 # tests
 # ----------------------------------------------------------------------------
@@ -143,6 +207,57 @@ def test_causal_limit_equals_sdpa():
     assert pin_causal_limit_sdpa()
     # the dense-cache workload's regime: k >= T, several frames
     assert pin_causal_limit_sdpa(M=9, n=3, k=40, T=5, H=3, D=8, seed=11)
+
+
+def test_transient_before_eviction_equals_sdpa():
+    assert pin_transient_before_eviction_is_sdpa()
+    assert pin_transient_before_eviction_is_sdpa(M=9, n=1, k=6, X=11, interval=3, seed=4)
+
+
+def test_transient_lse_counts_cache_and_own_tokens():
+    assert pin_transient_key_count()
+    assert pin_transient_key_count(n=3, k=2, X=14, interval=2)
+
+
+def test_keyframe_schedule_follows_the_walkthrough():
+    # scale frames always enter; then every interval-th frame counted from n
+    assert [gca.is_keyframe(x, n=3, interval=2) for x in range(9)] == \
+        [True, True, True, True, False, True, False, True, False]
+    assert all(gca.is_keyframe(x, n=3, interval=1) for x in range(20))
+    assert [gca.latest_keyframe(x, n=3, interval=2) for x in range(9)] == [0, 1, 2, 3, 3, 4, 4, 5, 5]
+
+
+@pytest.mark.parametrize("interval,anchor_block", [(2, False), (3, False), (2, True)])
+def test_keyframe_stream_equals_bruteforce(interval, anchor_block):
+    M, n, k, X, H, D = 4, 2, 3, 16, 2, 8
+    Q, K, V = _rand_stream(X, M, H, D, seed=13 + interval)
+    scale = 1 / math.sqrt(D)
+    keys = [y for y in range(X) if gca.is_keyframe(y, n=n, interval=interval)]
+    fkv = _frame_kv(K[keys], V[keys])
+    o2, l2 = gca.bruteforce_keyframes(Q, K, V, n=n, k=k, S=6, interval=interval, scale=scale,
+                                      anchor_block=anchor_block)
+    for x in range(X):
+        i = gca.latest_keyframe(x, n=n, interval=interval)
+        if gca.is_keyframe(x, n=n, interval=interval):
+            if anchor_block and i < n:
+                continue                     # the anchor block is one query block, not streamed
+            o, l = gca.stream_step(Q[x:x + 1], i, fkv, n=n, k=k, S=6, scale=scale,
+                                   anchor_block=anchor_block, impl="np")
+            o, l = o[0], l[0]
+        else:
+            o, l = gca.transient_step(Q[x], K[x], V[x], i, fkv, n=n, k=k, S=6, scale=scale,
+                                      anchor_block=anchor_block, impl="np")
+        assert np.abs(o - o2[x]).max() < 1e-12
+        assert np.abs(l - l2[x]).max() < 1e-12
+
+
+def test_transient_with_constant_values():
+    Q, K, V = _rand_stream(7, 5, 2, 8, seed=3)
+    V[:] = 2.5
+    keys = [0, 1, 2, 4, 6]
+    o, _ = gca.transient_step(Q[5], K[5], V[5], 3, _frame_kv(K[keys], V[keys]), n=2, k=2, S=6,
+                              scale=0.3, impl="np")
+    assert np.abs(o - 2.5).max() < 1e-12
 
 
 def test_single_frame_is_plain_attention():
@@ -380,3 +495,21 @@ def test_planted_future_frame_leak_is_caught(monkeypatch):
     monkeypatch.setattr(gca, "visible", wrong)
     assert not pin_mask_picture()
     assert not pin_causal_limit_sdpa()
+
+
+def test_planted_transient_without_own_tokens_is_caught(monkeypatch):
+    orig = gca.transient_step
+
+    def wrong(q, own_k, own_v, last_key, frame_kv, **kw):
+        return orig(q, own_k[:0], own_v[:0], last_key, frame_kv, **kw)
+    monkeypatch.setattr(gca, "transient_step", wrong)
+    assert not pin_transient_key_count()
+
+
+def test_planted_transient_reading_one_keyframe_late_is_caught(monkeypatch):
+    orig = gca.latest_keyframe
+
+    def wrong(x, *, n, interval):
+        return orig(x, n=n, interval=interval) - 1
+    monkeypatch.setattr(gca, "latest_keyframe", wrong)
+    assert not pin_transient_key_count()

@@ -16,7 +16,9 @@
 //   * eviction after frame t returns the image pages of every non-anchor frame
 //     f <= t-k (code walkthrough §2) — no bytes move;
 //   * the walk list is the image pages of the full frames some query frame of
-//     the block may see (ascending frame, then page), then every summary page.
+//     the block may see (ascending frame, then page), then every summary page;
+//   * ceil((S+M)/P) transient pages sit after the allocator's pages: a
+//     non-keyframe's K and V go there for one attention and are never kept.
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
@@ -49,6 +51,8 @@ struct gca_cache {
     int device = 0;
     int sms = 148;
     int P = 128, ipf = 1, num_pages = 0, Lq = 0;
+    int num_regular = 0;   // pages the allocator hands out; the transient pages follow
+    int tpf = 0;           // transient pages: ceil(Lq / P)
     size_t elem = 2;
     float scale = 0.f;
 
@@ -74,6 +78,9 @@ struct gca_cache {
     unsigned long long up_version = 0;
     int up_F = -1;
     int up_n = 0;
+    WalkEntry* d_walk_t = nullptr;   // walk list of the transient (non-keyframe) attention
+    unsigned long long tup_version = 0;
+    int tup_n = 0;
     float* ws_o = nullptr;
     float* ws_lse = nullptr;
     size_t ws_slots = 0;
@@ -98,6 +105,7 @@ void release(gca_cache* c) {
     cudaFree(c->kpool);
     cudaFree(c->vpool);
     cudaFree(c->d_walk);
+    cudaFree(c->d_walk_t);
     cudaFree(c->ws_o);
     cudaFree(c->ws_lse);
     cudaFree(c->st_k);
@@ -181,6 +189,96 @@ bool build_walk(const gca_cache* c, int F, std::vector<gca_page_entry_t>& out) {
     return true;
 }
 
+// Stages a walk list through the pinned ring and copies it to dst on st.
+int upload_walk(gca_cache* c, const std::vector<gca_page_entry_t>& w, WalkEntry* dst, cudaStream_t st) {
+    if ((int)w.size() > c->walk_cap) return GCA_ERR_CAPACITY;
+    const int slot = c->ring_pos;
+    c->ring_pos = (c->ring_pos + 1) % kRing;
+    if (cudaEventSynchronize(c->stage_ev[slot]) != cudaSuccess) return GCA_ERR_CUDA;
+    WalkEntry* hs = c->h_stage[slot];
+    for (size_t i = 0; i < w.size(); ++i) {
+        const gca_page_entry_t& e = w[i];
+        hs[i] = make_int4(e.page_id, e.n_valid, e.first, e.kind == GCA_PAGE_IMAGE ? e.frame : -1);
+    }
+    if (cudaMemcpyAsync(dst, hs, sizeof(WalkEntry) * w.size(), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaEventRecord(c->stage_ev[slot], st) != cudaSuccess)
+        return GCA_ERR_CUDA;
+    return GCA_OK;
+}
+
+// Attention of F query frames (the first is first_query_frame) over a device
+// walk list; stages host q / out / lse through the cache's buffers.
+int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query_frame,
+                  const WalkEntry* walk, int nwalk, void* out, float* lse, cudaStream_t st) {
+    const gca_config_t& g = c->cfg;
+    const int R = F * c->Lq;
+    const size_t qbytes = (size_t)R * g.num_heads * gca::kHeadDim * c->elem;
+    const void* qd = q;
+    if (!is_device_ptr(q)) {
+        if (cudaMemcpyAsync(c->st_q, q, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        qd = c->st_q;
+    }
+    const bool out_host = !is_device_ptr(out);
+    const bool lse_host = lse && !is_device_ptr(lse);
+
+    gca::AttendParams p{};
+    p.walk = walk;
+    p.nwalk = nwalk;
+    p.q = qd;
+    p.out = out_host ? c->st_out : out;
+    p.lse = lse ? (lse_host ? c->st_lse : lse) : nullptr;
+    p.R = R;
+    p.H = g.num_heads;
+    p.Lq = c->Lq;
+    p.first_query_frame = first_query_frame;
+    p.rule = {g.num_anchor, g.window, g.summary_tokens, g.anchor_block ? 1 : 0};
+    p.scale = c->scale;
+    p.scale_log2 = c->scale * 1.4426950408889634f;
+    p.layer = layer;
+    p.num_pages = c->num_pages;
+    p.P = c->P;
+    p.status = c->d_status;
+    p.ws_o = c->ws_o;
+    p.ws_lse = c->ws_lse;
+
+    cudaError_t err;
+    if (g.dtype == GCA_DTYPE_BF16) {
+        // split: QT query tiles x W workers over the head-major page stream
+        p.QT = ceil_div(R, kTileRows);
+        const long long total = (long long)g.num_heads * p.nwalk;
+        long long w = std::max(1, c->sms / ((p.QT + 1) / 2));   // CTAs = tile pairs x workers
+        w = std::min<long long>(w, (total + 3) / 4);
+        w = std::max<long long>(w, 1);
+        p.seg = ceil_div(total, w);
+        p.W = ceil_div(total, p.seg);
+        bool need_merge = false;
+        for (int h = 0; h < g.num_heads && !need_merge; ++h)
+            need_merge = ((long long)h * p.nwalk) / p.seg != ((long long)(h + 1) * p.nwalk - 1) / p.seg;
+        err = gca::launch_attend_sm100(c->tmK, c->tmV, p, st);
+        c->launches += 1;
+        if (err == cudaSuccess && need_merge) {
+            err = gca::launch_merge(p, st);
+            c->launches += 1;
+        }
+    } else {
+        p.QT = ceil_div(R, kTileRows);
+        p.W = 1;
+        p.seg = 1;
+        err = gca::launch_attend_f32(p, c->kpool, c->vpool, st);
+        c->launches += 1;
+    }
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return GCA_ERR_CUDA;
+    }
+    if (out_host && cudaMemcpyAsync(out, c->st_out, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GCA_ERR_CUDA;
+    if (lse_host && cudaMemcpyAsync(lse, c->st_lse, (size_t)R * g.num_heads * sizeof(float),
+                                    cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GCA_ERR_CUDA;
+    return GCA_OK;
+}
+
 int check_status(const gca_cache* c) {
     return (*(volatile int*)c->h_status) ? GCA_ERR_DEVICE_CHECK : GCA_OK;
 }
@@ -213,7 +311,8 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     if (g.head_dim != gca::kHeadDim || (g.page_size != 64 && g.page_size != 128) ||
         (g.dtype != GCA_DTYPE_BF16 && g.dtype != GCA_DTYPE_F32))
         return GCA_ERR_UNSUPPORTED;
-    if ((g.image_tokens + g.page_size - 1) / g.page_size > gca::kMaxImagePages)
+    // a frame's image pages, and a non-keyframe's transient pages, fit one append launch
+    if ((g.image_tokens + g.summary_tokens + g.page_size - 1) / g.page_size > gca::kMaxImagePages)
         return GCA_ERR_UNSUPPORTED;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
@@ -231,19 +330,22 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     const long long image_cap = (long long)(g.num_anchor + g.window + g.max_query_frames + g.frame_slack) * c->ipf;
     const long long summary_cap = ceil_div((long long)g.summary_tokens * g.max_frames, c->P);
     if (image_cap + summary_cap > (1LL << 30)) { delete c; return GCA_ERR_CAPACITY; }
-    c->num_pages = (int)(image_cap + summary_cap);
     c->Lq = g.image_tokens + g.summary_tokens;
+    c->num_regular = (int)(image_cap + summary_cap);
+    c->tpf = ceil_div(c->Lq, c->P);
+    c->num_pages = c->num_regular + c->tpf;
     c->elem = g.dtype == GCA_DTYPE_BF16 ? 2 : 4;
     c->scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.0f / sqrtf((float)g.head_dim);
     c->layer_frames.assign(g.num_layers, 0);
-    for (int i = 0; i < c->num_pages; ++i) c->free_pages.insert(i);
+    for (int i = 0; i < c->num_regular; ++i) c->free_pages.insert(i);
 
     const size_t tile = (size_t)c->P * gca::kHeadDim * c->elem;
     c->pool_bytes = (size_t)g.num_layers * c->num_pages * g.num_heads * tile;
     bool ok = cudaMalloc(&c->kpool, c->pool_bytes) == cudaSuccess &&
               cudaMalloc(&c->vpool, c->pool_bytes) == cudaSuccess;
     c->walk_cap = c->num_pages;
-    ok = ok && cudaMalloc(&c->d_walk, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess;
+    ok = ok && cudaMalloc(&c->d_walk, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
+         cudaMalloc(&c->d_walk_t, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess;
     for (int i = 0; ok && i < kRing; ++i) {
         ok = cudaHostAlloc((void**)&c->h_stage[i], sizeof(WalkEntry) * c->walk_cap, cudaHostAllocDefault) == cudaSuccess &&
              cudaEventCreateWithFlags(&c->stage_ev[i], cudaEventDisableTiming) == cudaSuccess;
@@ -402,7 +504,7 @@ int gca_evict_to_summary(gca_cache_t* c, int32_t* frames_evicted_out) {
 int gca_reset(gca_cache_t* c) {
     if (!c) return GCA_ERR_INVALID_ARG;
     c->free_pages.clear();
-    for (int i = 0; i < c->num_pages; ++i) c->free_pages.insert(i);
+    for (int i = 0; i < c->num_regular; ++i) c->free_pages.insert(i);
     c->image_pages.clear();
     c->summary_pages.clear();
     c->summary_opened_by.clear();
@@ -491,88 +593,77 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
     if (c->up_version != c->version || c->up_F != F) {
         std::vector<gca_page_entry_t> w;
         if (!build_walk(c, F, w)) return GCA_ERR_STATE;
-        const int slot = c->ring_pos;
-        c->ring_pos = (c->ring_pos + 1) % kRing;
-        if (cudaEventSynchronize(c->stage_ev[slot]) != cudaSuccess) return GCA_ERR_CUDA;
-        WalkEntry* hs = c->h_stage[slot];
-        for (size_t i = 0; i < w.size(); ++i) {
-            const gca_page_entry_t& e = w[i];
-            hs[i] = make_int4(e.page_id, e.n_valid, e.first, e.kind == GCA_PAGE_IMAGE ? e.frame : -1);
-        }
-        if (cudaMemcpyAsync(c->d_walk, hs, sizeof(WalkEntry) * w.size(), cudaMemcpyHostToDevice, st) != cudaSuccess ||
-            cudaEventRecord(c->stage_ev[slot], st) != cudaSuccess)
-            return GCA_ERR_CUDA;
+        if (int e = upload_walk(c, w, c->d_walk, st)) return e;
         c->up_version = c->version;
         c->up_F = F;
         c->up_n = (int)w.size();
     }
+    return run_attention(c, layer, q, F, c->T - F, c->d_walk, c->up_n, out, lse, st);
+}
 
-    const int R = F * c->Lq;
-    const size_t qbytes = (size_t)R * g.num_heads * gca::kHeadDim * c->elem;
-    const void* qd = q;
-    if (!is_device_ptr(q)) {
-        if (cudaMemcpyAsync(c->st_q, q, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        qd = c->st_q;
-    }
-    const bool out_host = !is_device_ptr(out);
-    const bool lse_host = lse && !is_device_ptr(lse);
+int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
+                         void* out, float* lse, void* stream) {
+    if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
+    const gca_config_t& g = c->cfg;
+    if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
+    if (c->layer_frames[layer] != c->T) return GCA_ERR_STATE;
+    if (int s = check_status(c)) return s;
+    DeviceGuard guard(c->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    gca::AttendParams p{};
-    p.walk = c->d_walk;
-    p.nwalk = c->up_n;
-    p.q = qd;
-    p.out = out_host ? c->st_out : out;
-    p.lse = lse ? (lse_host ? c->st_lse : lse) : nullptr;
-    p.R = R;
-    p.H = g.num_heads;
-    p.Lq = c->Lq;
-    p.first_query_frame = c->T - F;
-    p.rule = {g.num_anchor, g.window, g.summary_tokens, g.anchor_block ? 1 : 0};
-    p.scale = c->scale;
-    p.scale_log2 = c->scale * 1.4426950408889634f;
-    p.layer = layer;
-    p.num_pages = c->num_pages;
-    p.P = c->P;
-    p.status = c->d_status;
-    p.ws_o = c->ws_o;
-    p.ws_lse = c->ws_lse;
-
-    cudaError_t err;
-    if (g.dtype == GCA_DTYPE_BF16) {
-        // split: QT query tiles x W workers over the head-major page stream
-        p.QT = ceil_div(R, kTileRows);
-        const long long total = (long long)g.num_heads * p.nwalk;
-        long long w = std::max(1, c->sms / ((p.QT + 1) / 2));   // CTAs = tile pairs x workers
-        w = std::min<long long>(w, (total + 3) / 4);
-        w = std::max<long long>(w, 1);
-        p.seg = ceil_div(total, w);
-        p.W = ceil_div(total, p.seg);
-        bool need_merge = false;
-        for (int h = 0; h < g.num_heads && !need_merge; ++h)
-            need_merge = ((long long)h * p.nwalk) / p.seg != ((long long)(h + 1) * p.nwalk - 1) / p.seg;
-        err = gca::launch_attend_sm100(c->tmK, c->tmV, p, st);
-        c->launches += 1;
-        if (err == cudaSuccess && need_merge) {
-            err = gca::launch_merge(p, st);
-            c->launches += 1;
+    // The frame reads the cache as the latest keyframe t = T-1 does (query
+    // frame index t: its window and every summary), plus its own S+M tokens,
+    // which the walk list carries as full-frame pages of frame t.  With no
+    // keyframe yet it reads only itself.
+    const int i = c->T > 0 ? c->T - 1 : 0;
+    if (c->tup_version != c->version) {
+        std::vector<gca_page_entry_t> w;
+        if (c->T > 0 && !build_walk(c, 1, w)) return GCA_ERR_STATE;
+        for (int s = 0; s < c->tpf; ++s) {
+            const int first = s * c->P;
+            w.push_back({c->num_regular + s, GCA_PAGE_IMAGE, i, first, std::min(c->P, c->Lq - first)});
         }
-    } else {
-        p.QT = ceil_div(R, kTileRows);
-        p.W = 1;
-        p.seg = 1;
-        err = gca::launch_attend_f32(p, c->kpool, c->vpool, st);
-        c->launches += 1;
+        if (int e = upload_walk(c, w, c->d_walk_t, st)) return e;
+        c->tup_version = c->version;
+        c->tup_n = (int)w.size();
     }
-    if (err != cudaSuccess) {
+
+    // the frame's K and V into this layer's transient pages: token u of the
+    // frame (summary tokens first) at page u / P, slot u % P
+    gca::AppendParams p{};
+    const size_t bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
+    p.k = k;
+    p.v = v;
+    if (!is_device_ptr(k)) {
+        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        p.k = c->st_k;
+    }
+    if (!is_device_ptr(v)) {
+        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        p.v = c->st_v;
+    }
+    p.kpool = c->kpool;
+    p.vpool = c->vpool;
+    p.layer0 = layer;
+    p.nlayers = 1;
+    p.Lq = c->Lq;
+    p.S = 0;                 // every token of the frame is laid out like an image token
+    p.M = c->Lq;
+    p.H = g.num_heads;
+    p.P = c->P;
+    p.num_pages = c->num_pages;
+    p.elem_bytes = (int)c->elem;
+    p.sms = c->sms;
+    p.frame = i;
+    p.sum_seq0 = 0;
+    p.sum_page[0] = p.sum_page[1] = -1;
+    p.new_sum_seq = -1;
+    for (int s = 0; s < c->tpf; ++s) p.img_pages[s] = c->num_regular + s;
+    if (gca::launch_append(p, st) != cudaSuccess) {
         cudaGetLastError();
         return GCA_ERR_CUDA;
     }
-    if (out_host && cudaMemcpyAsync(out, c->st_out, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return GCA_ERR_CUDA;
-    if (lse_host && cudaMemcpyAsync(lse, c->st_lse, (size_t)R * g.num_heads * sizeof(float),
-                                    cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return GCA_ERR_CUDA;
-    return GCA_OK;
+    c->launches += 1;
+    return run_attention(c, layer, q, 1, i, c->d_walk_t, c->tup_n, out, lse, st);
 }
-
 }  // extern "C"
