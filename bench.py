@@ -489,6 +489,24 @@ def run_report(args):
                 cache.evict()
         cache.close()
 
+    # trajectory-memory variants on the 518x378 workload (one layer) at T=10000
+    for label, mode, n in (("camera token only", gca.GCA_MEMORY_CAMERA, None),
+                           ("sliding window (no memory, no anchors)", gca.GCA_MEMORY_NONE, 0)):
+        w = inputs.METRIC_518x378.with_(L=1) if n is None else inputs.METRIC_518x378.with_(L=1, n=n)
+        cache = gca.Cache.for_workload(w, max_frames=w.T, trajectory_memory=mode)
+        out = torch.empty((1, w.Lq, w.H, w.D), dtype=torch.bfloat16, device=dev)
+        for t in range(w.T):
+            cache.append(inputs.draw(w, t, "k", dev), inputs.draw(w, t, "v", dev))
+            cache.evict()
+        q = inputs.draw(w, w.T - 1, "q", dev)
+        att = _time_ms(lambda: cache.attend(0, q, out))
+        keys = cache.info().resident_tokens
+        fl = 4.0 * w.Lq * keys * w.H * w.D
+        print(json.dumps({"workload": w.name + " (layer 0 only)", "memory": label, "n": w.n, "T": w.T, "Lk": keys,
+                          "attend_ms": att, "tflops": fl / att / 1e9,
+                          "frac_bf16_peak": fl / att / 1e9 / pk["bf16"]}), flush=True)
+        cache.close()
+
     stream(inputs.WORKED_EXAMPLE, {100, 1000, 10000}, 10000)
     stream(inputs.DENSE_CAUSAL, {1000}, 1000)
     vo = inputs.WINDOWED_VO

@@ -64,6 +64,16 @@ typedef enum {
 } gca_status;
 
 typedef enum { GCA_DTYPE_BF16 = 0, GCA_DTYPE_F32 = 1 } gca_dtype;
+
+/* What a frame keeps once it leaves the window (its trajectory memory):
+ *   SUMMARY  all S special tokens (GCA; paper digest §2.2);
+ *   CAMERA   only special token 0, the camera token (the camera-only cache
+ *            option of code walkthrough §3.4);
+ *   NONE     nothing: with num_anchor = 0 this is the sliding-window mask of
+ *            the news article's mask figure (c).
+ * The special tokens a frame does not keep are stored with its image tokens
+ * and leave the cache with them. */
+typedef enum { GCA_MEMORY_SUMMARY = 0, GCA_MEMORY_CAMERA = 1, GCA_MEMORY_NONE = 2 } gca_memory;
 typedef enum { GCA_PAGE_IMAGE = 0, GCA_PAGE_SUMMARY = 1 } gca_page_kind;
 
 typedef struct gca_cache gca_cache_t;  /* opaque, library-owned */
@@ -87,12 +97,16 @@ typedef struct {
     int32_t max_query_frames; /* F_max >= 1: largest query block of gca_attend   */
     int32_t frame_slack;      /* extra full frames of page space (>= 0)          */
     float softmax_scale;      /* 0 selects 1/sqrt(D)                             */
+    int32_t trajectory_memory; /* gca_memory; 0 (SUMMARY) is GCA                 */
 } gca_config_t;
 
-/* One entry of the walk list (the pages gca_attend reads, in order).
+/* One entry of the walk list (the pages gca_attend reads, in order).  Below,
+ * s_k is the number of special tokens a frame keeps (S, 1 or 0 by
+ * trajectory_memory) and M' = M + S - s_k the tokens of a full frame's image
+ * pages (its unkept special tokens, then its M image tokens).
  * Image page: frame = owning frame, first = index of slot 0 among that frame's
- * image tokens.  Summary page: first = summary-stream index of slot 0 (token s
- * of frame t has stream index S*t+s), frame = first / S.
+ * M' image-page tokens.  Summary page: first = summary-stream index of slot 0
+ * (kept token s of frame t has stream index s_k*t+s), frame = first / s_k.
  * n_valid = tokens stored in the page. */
 typedef struct {
     int32_t page_id;
@@ -108,7 +122,7 @@ typedef struct {
     int32_t image_pages_per_frame;
     int32_t frames;           /* T: frames opened since create / reset           */
     int32_t full_frames;      /* frames still holding their image pages          */
-    int64_t resident_tokens;  /* M * full_frames + S * T                         */
+    int64_t resident_tokens;  /* M' * full_frames + s_k * T                      */
     void* k_pool;             /* device: [L][num_pages][H][P][D] of dtype        */
     void* v_pool;
     size_t pool_bytes;        /* bytes of one pool (all layers)                  */
@@ -117,8 +131,8 @@ typedef struct {
 } gca_info_t;
 
 /* Create a cache on CUDA device `device`.  Allocates both pools:
- * num_pages = (n + k + max_query_frames + frame_slack) * ceil(M/P)
- *           + ceil(S * max_frames / P)   pages the allocator hands out,
+ * num_pages = (n + k + max_query_frames + frame_slack) * ceil(M'/P)
+ *           + ceil(s_k * max_frames / P) pages the allocator hands out,
  *           + ceil((S+M) / P)            transient pages after them
  *                                        (gca_attend_transient), per layer.
  * Errors: INVALID_ARG (non-positive sizes, null out), UNSUPPORTED (head_dim
@@ -132,8 +146,8 @@ int gca_cache_destroy(gca_cache_t* cache);
 
 /* Append one frame's K and V (code walkthrough §2: each step adds the new
  * frame's M+S tokens).  layer == GCA_ALL_LAYERS or 0 opens frame T: the
- * allocator takes a summary page if the frame's summary tokens start a new one,
- * then ceil(M/P) image pages, smallest free page id first.  With
+ * allocator takes a summary page if the frame's s_k kept tokens start a new
+ * one, then ceil(M'/P) image pages, smallest free page id first.  With
  * GCA_ALL_LAYERS k and v are [L][S+M][H][D] and every layer is written in one
  * launch; otherwise they are [S+M][H][D] for that layer, and layers 1..L-1
  * must then append the open frame once each.  *frame_index_out (nullable)
@@ -145,16 +159,16 @@ int gca_append_frame(gca_cache_t* cache, int32_t layer, const void* k, const voi
 
 /* Compressing eviction (code walkthrough §2; paper-to-code article §2.3):
  * after frame t, every non-anchor frame f <= t-k that still holds image pages
- * returns them to the free set.  Its summary tokens stay in the summary stream,
- * so no bytes move.  Host-only, no stream.  *frames_evicted_out (nullable)
+ * returns them to the free set.  Its s_k kept tokens stay in the summary
+ * stream, so no bytes move.  Host-only, no stream.  *frames_evicted_out (nullable)
  * receives the number of frames reduced to summary tokens. */
 int gca_evict_to_summary(gca_cache_t* cache, int32_t* frames_evicted_out);
 
 /* GCA attention for one layer (paper digest §2.5): for the query block of the
  * F = num_query_frames most recent frames, q [F][S+M][H][D], query frame i
  * attends to
- *   every summary token of frames j <= i,
- *   every image token of frames j <= i with j < n or j >= i-k+1,
+ *   every kept special token (s < s_k) of frames j <= i,
+ *   every other token of frames j <= i with j < n or j >= i-k+1,
  *   and, with anchor_block, every token of frames j < n when i < n,
  * with softmax(scale * q.k) over those keys, fp32 accumulation.  out is
  * [F][S+M][H][D] in the cache dtype; lse (nullable) is [F][S+M][H] float32,

@@ -12,15 +12,17 @@ rules below are this project's own definition, stated once and implemented
 twice (here and in the C++ host code):
 
   * one pool of ``num_pages`` page ids, shared by every layer;
-  * frame t owns ceil(M/P) image pages holding its M image tokens in order;
-  * the S summary tokens of every frame go to one append-only summary stream:
-    token s of frame t has stream index S*t+s and lives in summary page
-    (S*t+s) // P, slot (S*t+s) % P;
+  * a frame keeps ``keep`` of its S special tokens as trajectory memory (S by
+    default; 1 = the camera token only; 0 = none, the sliding-window cache):
+    they go to one append-only summary stream, token s < keep of frame t at
+    stream index keep*t+s, summary page (keep*t+s) // P, slot (keep*t+s) % P;
+  * frame t owns ceil(M'/P) image pages, M' = M + S - keep, holding its other
+    special tokens and then its M image tokens in token order (slot tau-keep);
   * pages are taken smallest free id first, in token order within a frame:
     a new summary page (when the frame's summary tokens cross a page
     boundary) before the frame's image pages;
-  * capacity: (n + k + max_query_frames + frame_slack) * ceil(M/P) image pages
-    plus ceil(S*max_frames/P) summary pages;
+  * capacity: (n + k + max_query_frames + frame_slack) * ceil(M'/P) image pages
+    plus ceil(keep*max_frames/P) summary pages;
   * evict (after frame t): every non-anchor frame f <= t-k still holding image
     pages returns them to the free set; its summary tokens stay where they are,
     so eviction moves no bytes;
@@ -30,8 +32,8 @@ twice (here and in the C++ host code):
     order and page order, then every summary page in stream order.  Each entry
     is (page_id, kind, frame, first, n_valid): kind 0 = image, 1 = summary;
     for an image page ``frame`` is its frame and ``first`` the index of its
-    slot 0 among the frame's image tokens; for a summary page ``first`` is the
-    stream index of slot 0 and ``frame`` = first // S.
+    slot 0 among the frame's M' image-page tokens; for a summary page ``first``
+    is the stream index of slot 0 and ``frame`` = first // keep.
 """
 from __future__ import annotations
 
@@ -52,13 +54,15 @@ class StateError(RuntimeError):
 class PageTableSim:
     def __init__(self, *, M: int, S: int, P: int, n: int, k: int, max_frames: int,
                  max_query_frames: int = 1, frame_slack: int = 0,
-                 anchor_block: bool = False):
+                 anchor_block: bool = False, keep: int = None):
         self.M, self.S, self.P, self.n, self.k = M, S, P, n, k
+        self.keep = S if keep is None else keep     # special tokens kept per frame
+        self.Mi = M + S - self.keep                  # tokens of a full frame's image pages
         self.max_frames = max_frames
         self.anchor_block = anchor_block
-        self.ipf = math.ceil(M / P)
+        self.ipf = math.ceil(self.Mi / P)
         self.image_capacity = (n + k + max_query_frames + frame_slack) * self.ipf
-        self.summary_capacity = math.ceil(S * max_frames / P)
+        self.summary_capacity = math.ceil(self.keep * max_frames / P)
         self.num_pages = self.image_capacity + self.summary_capacity
         self.reset()
 
@@ -77,11 +81,12 @@ class PageTableSim:
         t = self.T
         if t >= self.max_frames:
             raise CapacityError("max_frames reached")
-        new_summary = sum(1 for s in range(self.S) if (self.S * t + s) % self.P == 0)
+        kp = self.keep
+        new_summary = sum(1 for s in range(kp) if (kp * t + s) % self.P == 0)
         if len(self.free) < self.ipf + new_summary:
             raise CapacityError("page pool exhausted")
-        for s in range(self.S):
-            if (self.S * t + s) % self.P == 0:
+        for s in range(kp):
+            if (kp * t + s) % self.P == 0:
                 self.summary_pages.append(self._take())
         self.image_pages[t] = [self._take() for _ in range(self.ipf)]
         self.T += 1
@@ -115,21 +120,21 @@ class PageTableSim:
             if any(self._frame_seen(i, f) for i in queries):
                 for seq, pid in enumerate(self.image_pages[f]):
                     first = seq * self.P
-                    out.append((pid, IMAGE, f, first, min(self.P, self.M - first)))
-        total = self.S * self.T
+                    out.append((pid, IMAGE, f, first, min(self.P, self.Mi - first)))
+        total = self.keep * self.T
         for seq, pid in enumerate(self.summary_pages):
             first = seq * self.P
-            out.append((pid, SUMMARY, first // self.S, first, min(self.P, total - first)))
+            out.append((pid, SUMMARY, first // self.keep, first, min(self.P, total - first)))
         return out
 
     def resident_tokens(self) -> int:
-        """Tokens held: image tokens of full frames plus every summary token."""
-        return self.M * len(self.image_pages) + self.S * self.T
+        """Tokens held: image-page tokens of full frames plus every kept token."""
+        return self.Mi * len(self.image_pages) + self.keep * self.T
 
     def slot_of(self, frame: int, tau: int):
-        """(page id, slot) of token slot tau of a frame (tau < S: summary)."""
-        if tau < self.S:
-            idx = self.S * frame + tau
+        """(page id, slot) of token slot tau of a frame (tau < keep: summary stream)."""
+        if tau < self.keep:
+            idx = self.keep * frame + tau
             return self.summary_pages[idx // self.P], idx % self.P
-        m = tau - self.S
+        m = tau - self.keep
         return self.image_pages[frame][m // self.P], m % self.P

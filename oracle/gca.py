@@ -57,11 +57,14 @@ LIB_PATH = os.path.join(HERE, "liboracle.so")
 # ----------------------------------------------------------------------------
 # closed forms (paper digest §2.4)
 # ----------------------------------------------------------------------------
-def cache_tokens(M: int, S: int, n: int, k: int, T: int) -> int:
+def cache_tokens(M: int, S: int, n: int, k: int, T: int, keep: Optional[int] = None) -> int:
     """Tokens cached by GCA after T frames: full frames hold M image tokens,
     every frame holds S summary tokens.  Full frames are the first
-    min(T, n+k) frames' worth: n anchors plus the k-frame window."""
-    return M * min(T, n + k) + S * T
+    min(T, n+k) frames' worth: n anchors plus the k-frame window.  With
+    ``keep`` < S special tokens kept per frame (camera-only: 1; none: 0) a
+    full frame holds its other S-keep special tokens with its image tokens."""
+    kp = S if keep is None else keep
+    return (M + S - kp) * min(T, n + k) + kp * T
 
 
 def causal_tokens(M: int, S: int, T: int) -> int:
@@ -73,19 +76,22 @@ def causal_tokens(M: int, S: int, T: int) -> int:
 # (O2) token-level visibility predicate, paper digest §2.5
 # ----------------------------------------------------------------------------
 def visible(i: int, j: int, tau: int, *, n: int, k: int, S: int,
-            anchor_block: bool = False) -> bool:
+            anchor_block: bool = False, keep: Optional[int] = None) -> bool:
     """May a query token of frame i attend to token slot tau of frame j?
 
     Slots 0..S-1 are the summary tokens (camera, anchor, 4 registers), slots
-    S..S+M-1 the image tokens.  Frame i itself is part of its window.
+    S..S+M-1 the image tokens.  Frame i itself is part of its window.  The
+    first ``keep`` slots (default all S) form the trajectory memory; the other
+    special tokens are seen only while the frame is full, like image tokens.
     """
+    kp = S if keep is None else keep
     if anchor_block and i < n and j < n:
         return True                       # anchors attend jointly (one block)
     if j > i:
         return False                      # no future frames
-    if tau < S:
-        return True                       # summary tokens of every earlier frame
-    return j < n or j >= i - k + 1        # image tokens: anchors and the window
+    if tau < kp:
+        return True                       # kept tokens of every earlier frame
+    return j < n or j >= i - k + 1        # the rest: anchors and the window
 
 
 # ----------------------------------------------------------------------------
@@ -119,8 +125,11 @@ shape [S+M][H][D], or [S][H][D] when summary_only."""
 
 
 def gather_keys(i: int, frame_kv: FrameKV, *, n: int, k: int, S: int,
-                anchor_block: bool = False):
-    """Keys and values that query frame i attends to, [Nk][H][D] float32."""
+                anchor_block: bool = False, keep: Optional[int] = None):
+    """Keys and values that query frame i attends to, [Nk][H][D] float32.
+    Frames reduced to their trajectory memory contribute their first ``keep``
+    (default S) tokens."""
+    kp = S if keep is None else keep
     full, summary = stream_state(i, n=n, k=k, anchor_block=anchor_block)
     ks, vs = [], []
     for f in full:
@@ -129,8 +138,8 @@ def gather_keys(i: int, frame_kv: FrameKV, *, n: int, k: int, S: int,
         vs.append(vf)
     for f in summary:
         kf, vf = frame_kv(f, True)
-        ks.append(kf[:S])
-        vs.append(vf[:S])
+        ks.append(kf[:kp])
+        vs.append(vf[:kp])
     return np.concatenate(ks, 0), np.concatenate(vs, 0)
 
 
@@ -213,7 +222,7 @@ def attention(q, k, v, scale, impl: str = "c"):
 # ----------------------------------------------------------------------------
 def stream_step(q_block: np.ndarray, last_frame: int, frame_kv: FrameKV, *, n: int,
                 k: int, S: int, scale: float, anchor_block: bool = False,
-                rows: Optional[Sequence[int]] = None, impl: str = "c"):
+                rows: Optional[Sequence[int]] = None, impl: str = "c", keep: Optional[int] = None):
     """GCA output of the query block that ends at frame ``last_frame``.
 
     q_block is [F][S+M][H][D] (the F most recent frames' queries).  Returns
@@ -224,7 +233,7 @@ def stream_step(q_block: np.ndarray, last_frame: int, frame_kv: FrameKV, *, n: i
     outs, lses = [], []
     for b in range(F):
         i = last_frame - F + 1 + b
-        kk, vv = gather_keys(i, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block)
+        kk, vv = gather_keys(i, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
         qi = q_block[b] if rows is None else q_block[b][list(rows)]
         o, l = attention(qi, kk, vv, scale, impl)
         outs.append(o)
@@ -251,7 +260,7 @@ def latest_keyframe(x: int, *, n: int, interval: int) -> int:
 def transient_step(q: np.ndarray, own_k: np.ndarray, own_v: np.ndarray, last_key: int,
                    frame_kv: FrameKV, *, n: int, k: int, S: int, scale: float,
                    anchor_block: bool = False, rows: Optional[Sequence[int]] = None,
-                   impl: str = "c"):
+                   impl: str = "c", keep: Optional[int] = None):
     """Output of a non-keyframe, q / own_k / own_v [S+M][H][D].
 
     The frame is predicted like every other frame but its K/V never enters the
@@ -262,7 +271,8 @@ def transient_step(q: np.ndarray, own_k: np.ndarray, own_v: np.ndarray, last_key
     """
     ks, vs = [], []
     if last_key >= 0:
-        kk, vv = gather_keys(last_key, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block)
+        kk, vv = gather_keys(last_key, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block,
+                             keep=keep)
         ks.append(kk)
         vs.append(vv)
     ks.append(own_k)
@@ -272,7 +282,8 @@ def transient_step(q: np.ndarray, own_k: np.ndarray, own_v: np.ndarray, last_key
 
 
 def bruteforce_keyframes(Q: np.ndarray, K: np.ndarray, V: np.ndarray, *, n: int, k: int,
-                         S: int, interval: int, scale: float, anchor_block: bool = False):
+                         S: int, interval: int, scale: float, anchor_block: bool = False,
+                         keep: Optional[int] = None):
     """Every video frame's output at once for a stream in which only keyframes
     are cached.  Q, K, V [X][S+M][H][D] over all X video frames.  A query of
     frame x sees token tau of keyframe y when the token rule allows it between
@@ -295,7 +306,7 @@ def bruteforce_keyframes(Q: np.ndarray, K: np.ndarray, V: np.ndarray, *, n: int,
             for tau in range(Lq):
                 if y in kid and i >= 0:
                     vis[y * Lq + tau] = visible(i, kid[y], tau, n=n, k=k, S=S,
-                                                anchor_block=anchor_block)
+                                                anchor_block=anchor_block, keep=keep)
                 if y == x and x not in kid:
                     vis[y * Lq + tau] = True
         o, l = attention_np(q[x], kf[vis], vf[vis], scale)
@@ -308,25 +319,26 @@ def bruteforce_keyframes(Q: np.ndarray, K: np.ndarray, V: np.ndarray, *, n: int,
 # (O2) brute force over the whole sequence with an explicit mask
 # ----------------------------------------------------------------------------
 def visibility_mask(T: int, Lq: int, *, n: int, k: int, S: int,
-                    anchor_block: bool = False) -> np.ndarray:
+                    anchor_block: bool = False, keep: Optional[int] = None) -> np.ndarray:
     """Boolean [T*Lq][T*Lq] mask of the whole stream from the token rule."""
     keys = [(j, tau) for j in range(T) for tau in range(Lq)]
     frame_rows = np.zeros((T, T * Lq), dtype=bool)
     for i in range(T):
         for b, (j, tau) in enumerate(keys):
-            frame_rows[i, b] = visible(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block)
+            frame_rows[i, b] = visible(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block,
+                                       keep=keep)
     return np.repeat(frame_rows, Lq, axis=0)
 
 
 def bruteforce(Q: np.ndarray, K: np.ndarray, V: np.ndarray, *, n: int, k: int, S: int,
-               scale: float, anchor_block: bool = False):
+               scale: float, anchor_block: bool = False, keep: Optional[int] = None):
     """Every frame's GCA output at once: Q, K, V [T][S+M][H][D] -> out
     [T][S+M][H][D], lse [T][S+M][H] (float64)."""
     T, Lq, H, D = Q.shape
     q = Q.reshape(T * Lq, H, D).astype(np.float64)
     kx = K.reshape(T * Lq, H, D).astype(np.float64)
     vx = V.reshape(T * Lq, H, D).astype(np.float64)
-    mask = visibility_mask(T, Lq, n=n, k=k, S=S, anchor_block=anchor_block)
+    mask = visibility_mask(T, Lq, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
     s = scale * np.einsum("rhd,uhd->hru", q, kx)
     s = np.where(mask[None], s, -np.inf)
     mx = s.max(axis=2, keepdims=True)

@@ -60,13 +60,14 @@ def needed_full(w: inputs.Workload, t: int, F: int = 1):
 
 
 def oracle_step(mirror: Mirror, layer: int, q_block: np.ndarray, last: int, F: int = 1,
-                rows=None, anchor_block: bool = False):
+                rows=None, anchor_block: bool = False, keep=None):
     """Oracle output of a query block; q_block holds all heads, the mirror's
-    head subset (if any) is applied to it."""
+    head subset (if any) is applied to it.  keep: special tokens a frame keeps
+    after eviction (default all S)."""
     w = mirror.w
     qb = q_block if mirror.heads is None else q_block[:, :, mirror.heads]
     return ogca.stream_step(qb, last, mirror.frame_kv(layer), n=w.n, k=w.k, S=w.S,
-                            scale=w.softmax_scale, anchor_block=anchor_block, rows=rows)
+                            scale=w.softmax_scale, anchor_block=anchor_block, rows=rows, keep=keep)
 
 
 def oracle_transient(mirror: Mirror, layer: int, q: np.ndarray, k: np.ndarray, v: np.ndarray,

@@ -64,15 +64,26 @@ def test_tiny_stream_every_step(w):
     print(f"{w.name}: max |dO| {max(e[0] for e in errs):.3e}, max |dlse| {max(e[1] for e in errs):.3e}")
 
 
+MEMORY = {"summary": (gca.GCA_MEMORY_SUMMARY, 6, None), "camera": (gca.GCA_MEMORY_CAMERA, 1, None),
+          "none_n0": (gca.GCA_MEMORY_NONE, 0, 0)}
+
+
+@pytest.mark.parametrize("memory", list(MEMORY))
 @pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
-def test_append_writes_pool_bytes_bit_exact(w):
-    cache = gca.Cache.for_workload(w)
+def test_append_writes_pool_bytes_bit_exact(w, memory):
+    mode, keep, n = MEMORY[memory]
+    if n is not None:
+        w = w.with_(n=n)
+    cache = gca.Cache.for_workload(w, trajectory_memory=mode)
+    sim = _sim(w, keep=keep)
     frames = {}
     for t in range(w.T):
         k = inputs.draw(w, t, "k").cuda()
         v = inputs.draw(w, t, "v").cuda()
         cache.append(k, v)
-        cache.evict()
+        sim.append()
+        assert cache.evict() == sim.evict()
+        assert cache.layout() == sim.walk()
         frames[t] = (k[0].cpu(), v[0].cpu())
     torch.cuda.synchronize()
     info = cache.info()
@@ -84,8 +95,9 @@ def test_append_writes_pool_bytes_bit_exact(w):
                 try:
                     pid, slot = cache.token_slot(t, tau)
                 except gca.GCAError as e:
-                    assert e.name == "GCA_ERR_STATE" and tau >= w.S   # evicted image token
+                    assert e.name == "GCA_ERR_STATE" and tau >= keep   # left with the image pages
                     continue
+                assert (pid, slot) == sim.slot_of(t, tau)
                 got = pool[0, pid, :, slot, :]
                 assert torch.equal(got.view(torch.int16 if w.dtype == "bf16" else torch.int32),
                                    kv[idx][tau].view(torch.int16 if w.dtype == "bf16" else torch.int32))
@@ -263,6 +275,34 @@ def test_page_size_64():
         want, _ = oracle_step(mirror, 0, q.float().cpu().numpy(), t)
         torch.cuda.synchronize()
         assert max_err(out, want) <= TOL["bf16"], t
+
+
+# ----------------------------------------------------------------------------
+# trajectory-memory variants: camera token only; none (sliding window, n = 0)
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("memory", ["camera", "none_n0"])
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16], ids=["f32", "bf16"])
+def test_memory_variant_stream_every_step(w, memory):
+    mode, keep, n = MEMORY[memory]
+    if n is not None:
+        w = w.with_(n=n)
+    cache = gca.Cache.for_workload(w, trajectory_memory=mode)
+    sim = _sim(w, keep=keep)
+    mirror = Mirror(w, [0])
+    for t in range(w.T):
+        k, v, q = (inputs.draw(w, t, x).cuda() for x in "kvq")
+        assert cache.append(k, v) == t
+        sim.append()
+        mirror.record(t, k, v, keep_full=True)
+        assert cache.evict() == sim.evict()
+        assert cache.layout() == sim.walk()
+        assert cache.info().resident_tokens == sim.resident_tokens()
+        out, lse = attend(cache, 0, q[0:1].contiguous())
+        want, wlse = oracle_step(mirror, 0, q[0:1].float().cpu().numpy(), t, keep=keep)
+        torch.cuda.synchronize()
+        assert max_err(out[0], want[0]) <= TOL[w.dtype], t
+        assert max_err(lse[0], wlse[0]) <= LSE_TOL[w.dtype], t
+    assert cache.status() == 0
 
 
 # ----------------------------------------------------------------------------

@@ -176,6 +176,45 @@ def pin_transient_key_count(M=5, S=6, n=2, k=3, X=17, interval=3, H=1, D=8):
     return True
 
 
+def pin_sliding_window_is_banded_sdpa(M=5, k=3, T=9, H=2, D=16, seed=17):
+    """No anchors and no trajectory memory (keep = 0): frame i sees every token
+    of frames i-k+1..i and nothing else — the sliding-window mask of the mask
+    figure (c), here an explicit frame band through torch SDPA (fp64)."""
+    Q, K, V = _rand_stream(T, M, H, D, seed)
+    scale = 1 / math.sqrt(D)
+    Lq = M + 6
+    q = torch.from_numpy(Q.astype(np.float64)).reshape(T * Lq, H, D).permute(1, 0, 2)
+    kk = torch.from_numpy(K.astype(np.float64)).reshape(T * Lq, H, D).permute(1, 0, 2)
+    vv = torch.from_numpy(V.astype(np.float64)).reshape(T * Lq, H, D).permute(1, 0, 2)
+    fr = torch.arange(T).repeat_interleave(Lq)
+    band = (fr[None, :] <= fr[:, None]) & (fr[None, :] >= fr[:, None] - k + 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q[None], kk[None], vv[None], attn_mask=band,
+                                                           scale=scale)
+    ref = ref[0].permute(1, 0, 2).reshape(T, Lq, H, D).numpy()
+    o1 = []
+    for i in range(T):
+        o, _ = gca.stream_step(Q[i:i + 1], i, _frame_kv(K, V), n=0, k=k, S=6, scale=scale,
+                               impl="np", keep=0)
+        o1.append(o[0])
+    o2, _ = gca.bruteforce(Q, K, V, n=0, k=k, S=6, scale=scale, keep=0)
+    return bool(np.abs(np.stack(o1) - ref).max() < 1e-12 and np.abs(o2 - ref).max() < 1e-12)
+
+
+def pin_camera_only_key_count(M=5, S=6, n=2, k=3, T=12, H=1, D=8):
+    """Camera-only memory (keep = 1), Q = 0: lse = ln(#keys), and #keys is every
+    token of the min(T, n+k) full frames plus one camera token per other frame."""
+    Q, K, V = _rand_stream(T, M, H, D, seed=29, S=S)
+    Q[:] = 0
+    for i in range(T):
+        _, lse = gca.stream_step(Q[i:i + 1], i, _frame_kv(K, V), n=n, k=k, S=S, scale=0.125,
+                                 impl="np", keep=1)
+        full = min(i + 1, n + k)
+        want = math.log((M + S) * full + (i + 1 - full))
+        if not np.allclose(lse[0], want, atol=1e-12, rtol=0):
+            return False
+    return True
+
+
 # ----------------------------------------------------------------------------
 # tests
 # ----------------------------------------------------------------------------
@@ -258,6 +297,56 @@ def test_transient_with_constant_values():
     o, _ = gca.transient_step(Q[5], K[5], V[5], 3, _frame_kv(K[keys], V[keys]), n=2, k=2, S=6,
                               scale=0.3, impl="np")
     assert np.abs(o - 2.5).max() < 1e-12
+
+
+def test_sliding_window_mask_equals_banded_sdpa():
+    assert pin_sliding_window_is_banded_sdpa()
+    assert pin_sliding_window_is_banded_sdpa(M=3, k=1, T=5, seed=2)
+
+
+def test_camera_only_key_count():
+    assert pin_camera_only_key_count()
+    assert pin_camera_only_key_count(n=0, k=2, T=9)
+    # the closed form agrees with the per-step count
+    for T in (1, 5, 40):
+        assert gca.cache_tokens(500, 6, 3, 16, T, keep=1) == 505 * min(T, 19) + T
+        assert gca.cache_tokens(500, 6, 0, 16, T, keep=0) == 506 * min(T, 16)
+
+
+@pytest.mark.parametrize("keep,n,anchor_block", [(1, 2, False), (0, 2, False), (1, 2, True), (0, 0, False)])
+def test_memory_variants_stream_equals_bruteforce(keep, n, anchor_block):
+    M, k, T, H, D = 4, 3, 10, 2, 8
+    Q, K, V = _rand_stream(T, M, H, D, seed=31 + keep)
+    scale = 1 / math.sqrt(D)
+    o2, l2 = gca.bruteforce(Q, K, V, n=n, k=k, S=6, scale=scale, anchor_block=anchor_block, keep=keep)
+    for i in range(T):
+        if anchor_block and i < n:
+            continue
+        o, l = gca.stream_step(Q[i:i + 1], i, _frame_kv(K, V), n=n, k=k, S=6, scale=scale,
+                               anchor_block=anchor_block, impl="np", keep=keep)
+        assert np.abs(o[0] - o2[i]).max() < 1e-12
+        assert np.abs(l[0] - l2[i]).max() < 1e-12
+
+
+@pytest.mark.parametrize("keep", [6, 1, 0])
+def test_allocator_memory_variants_follow_closed_form(keep):
+    n = 0 if keep == 0 else 3
+    sim = PageTableSim(M=500, S=6, P=128, n=n, k=16, max_frames=400, keep=keep)
+    for T in range(1, 401):
+        sim.append()
+        sim.evict()
+        want = gca.cache_tokens(500, 6, n, 16, T, keep=keep)
+        assert sim.resident_tokens() == want
+        assert sum(e[4] for e in sim.walk()) == want
+    assert sim.ipf == math.ceil((500 + 6 - keep) / 128)
+    # token slots: kept tokens in the stream, the others in the frame's image pages in order
+    t = 399
+    for tau in range(506):
+        pid, slot = sim.slot_of(t, tau)
+        if tau < keep:
+            assert pid in sim.summary_pages and slot == (keep * t + tau) % 128
+        else:
+            assert pid == sim.image_pages[t][(tau - keep) // 128] and slot == (tau - keep) % 128
 
 
 def test_single_frame_is_plain_attention():
@@ -445,10 +534,10 @@ def test_allocator_reset_matches_fresh_windowed_stream():
 def test_planted_window_off_by_one_is_caught(monkeypatch):
     orig = gca.visible
 
-    def wrong(i, j, tau, *, n, k, S, anchor_block=False):
+    def wrong(i, j, tau, *, n, k, S, anchor_block=False, keep=None):
         if tau >= S and j <= i and j >= n:
             return j >= i - k             # window one frame too wide
-        return orig(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block)
+        return orig(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
     monkeypatch.setattr(gca, "visible", wrong)
     assert not pin_mask_picture()
 
@@ -488,10 +577,10 @@ def test_planted_swapped_operands_are_caught(monkeypatch):
 def test_planted_future_frame_leak_is_caught(monkeypatch):
     orig = gca.visible
 
-    def wrong(i, j, tau, *, n, k, S, anchor_block=False):
+    def wrong(i, j, tau, *, n, k, S, anchor_block=False, keep=None):
         if j == i + 1 and tau < S:
             return True
-        return orig(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block)
+        return orig(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
     monkeypatch.setattr(gca, "visible", wrong)
     assert not pin_mask_picture()
     assert not pin_causal_limit_sdpa()
@@ -513,3 +602,23 @@ def test_planted_transient_reading_one_keyframe_late_is_caught(monkeypatch):
         return orig(x, n=n, interval=interval) - 1
     monkeypatch.setattr(gca, "latest_keyframe", wrong)
     assert not pin_transient_key_count()
+
+
+def test_planted_camera_only_keeping_every_summary_token_is_caught(monkeypatch):
+    orig = gca.gather_keys
+
+    def wrong(i, frame_kv, *, n, k, S, anchor_block=False, keep=None):
+        return orig(i, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block, keep=None)
+    monkeypatch.setattr(gca, "gather_keys", wrong)
+    assert not pin_camera_only_key_count()
+
+
+def test_planted_sliding_window_with_anchor_leak_is_caught(monkeypatch):
+    orig = gca.visible
+
+    def wrong(i, j, tau, *, n, k, S, anchor_block=False, keep=None):
+        if j == 0 and j <= i:
+            return True                   # frame 0 treated as an anchor
+        return orig(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
+    monkeypatch.setattr(gca, "visible", wrong)
+    assert not pin_sliding_window_is_banded_sdpa()

@@ -11,8 +11,12 @@
 //   * pages are taken smallest free id first, in token order within a frame:
 //     a new summary page when the frame's summary tokens reach one, then the
 //     frame's ceil(M/P) image pages;
-//   * summary token s of frame t sits at stream index S*t+s, page
-//     (S*t+s)/P of the summary stream, slot (S*t+s)%P;
+//   * the first `keep` special tokens of a frame form its trajectory memory
+//     (keep = S by default; 1 keeps only the camera token; 0 keeps nothing):
+//     token s < keep of frame t sits at stream index keep*t+s, page
+//     (keep*t+s)/P of the summary stream, slot (keep*t+s)%P; the frame's other
+//     S-keep special tokens and its M image tokens fill its image pages, in
+//     token order (slot tau-keep), and leave with them at eviction;
 //   * eviction after frame t returns the image pages of every non-anchor frame
 //     f <= t-k (code walkthrough §2) — no bytes move;
 //   * the walk list is the image pages of the full frames some query frame of
@@ -51,6 +55,8 @@ struct gca_cache {
     int device = 0;
     int sms = 148;
     int P = 128, ipf = 1, num_pages = 0, Lq = 0;
+    int keep = 0;          // special tokens per frame kept in the summary stream
+    int ftok = 0;          // tokens in a full frame's image pages: Lq - keep
     int num_regular = 0;   // pages the allocator hands out; the transient pages follow
     int tpf = 0;           // transient pages: ceil(Lq / P)
     size_t elem = 2;
@@ -177,13 +183,13 @@ bool build_walk(const gca_cache* c, int F, std::vector<gca_page_entry_t>& out) {
         for (size_t s = 0; s < kv.second.size(); ++s) {
             const int first = (int)s * c->P;
             out.push_back({kv.second[s], GCA_PAGE_IMAGE, kv.first, first,
-                           std::min(c->P, c->cfg.image_tokens - first)});
+                           std::min(c->P, c->ftok - first)});
         }
     }
-    const long long total = (long long)c->cfg.summary_tokens * c->T;
+    const long long total = (long long)c->keep * c->T;
     for (size_t s = 0; s < c->summary_pages.size(); ++s) {
         const int first = (int)s * c->P;
-        out.push_back({c->summary_pages[s], GCA_PAGE_SUMMARY, first / c->cfg.summary_tokens, first,
+        out.push_back({c->summary_pages[s], GCA_PAGE_SUMMARY, first / c->keep, first,
                        (int)std::min<long long>(c->P, total - first)});
     }
     return true;
@@ -231,7 +237,7 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     p.H = g.num_heads;
     p.Lq = c->Lq;
     p.first_query_frame = first_query_frame;
-    p.rule = {g.num_anchor, g.window, g.summary_tokens, g.anchor_block ? 1 : 0};
+    p.rule = {g.num_anchor, g.window, c->keep, g.anchor_block ? 1 : 0};
     p.scale = c->scale;
     p.scale_log2 = c->scale * 1.4426950408889634f;
     p.layer = layer;
@@ -306,7 +312,8 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     const gca_config_t& g = *cfg;
     if (g.num_layers < 1 || g.num_heads < 1 || g.image_tokens < 1 || g.summary_tokens < 1 ||
         g.num_anchor < 0 || g.window < 1 || g.max_frames < 1 || g.max_query_frames < 1 ||
-        g.frame_slack < 0 || g.softmax_scale < 0.f)
+        g.frame_slack < 0 || g.softmax_scale < 0.f || g.trajectory_memory < GCA_MEMORY_SUMMARY ||
+        g.trajectory_memory > GCA_MEMORY_NONE)
         return GCA_ERR_INVALID_ARG;
     if (g.head_dim != gca::kHeadDim || (g.page_size != 64 && g.page_size != 128) ||
         (g.dtype != GCA_DTYPE_BF16 && g.dtype != GCA_DTYPE_F32))
@@ -326,9 +333,12 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     c->device = device;
     cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, device);
     c->P = g.page_size;
-    c->ipf = ceil_div(g.image_tokens, c->P);
+    c->keep = g.trajectory_memory == GCA_MEMORY_SUMMARY ? g.summary_tokens
+            : g.trajectory_memory == GCA_MEMORY_CAMERA ? 1 : 0;
+    c->ftok = g.image_tokens + g.summary_tokens - c->keep;
+    c->ipf = ceil_div(c->ftok, c->P);
     const long long image_cap = (long long)(g.num_anchor + g.window + g.max_query_frames + g.frame_slack) * c->ipf;
-    const long long summary_cap = ceil_div((long long)g.summary_tokens * g.max_frames, c->P);
+    const long long summary_cap = ceil_div((long long)c->keep * g.max_frames, c->P);
     if (image_cap + summary_cap > (1LL << 30)) { delete c; return GCA_ERR_CAPACITY; }
     c->Lq = g.image_tokens + g.summary_tokens;
     c->num_regular = (int)(image_cap + summary_cap);
@@ -410,7 +420,7 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
             if (c->layer_frames[l] != c->T) return GCA_ERR_STATE;
         if (c->T >= g.max_frames) return GCA_ERR_CAPACITY;
         t = c->T;
-        const int S = g.summary_tokens;
+        const int S = c->keep;
         int new_sum = 0;
         for (int s = 0; s < S; ++s) new_sum += ((S * t + s) % c->P) == 0;
         if ((int)c->free_pages.size() < c->ipf + new_sum) return GCA_ERR_CAPACITY;
@@ -455,17 +465,17 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
     p.layer0 = l0;
     p.nlayers = nl;
     p.Lq = c->Lq;
-    p.S = g.summary_tokens;
-    p.M = g.image_tokens;
+    p.S = c->keep;           // tokens s < keep go to the summary stream,
+    p.M = c->ftok;           // the rest to the frame's image pages
     p.H = g.num_heads;
     p.P = c->P;
     p.num_pages = c->num_pages;
     p.elem_bytes = (int)c->elem;
     p.sms = c->sms;
     p.frame = t;
-    const int S = g.summary_tokens;
+    const int S = c->keep;
     p.sum_seq0 = (S * t) / c->P;
-    p.sum_page[0] = c->summary_pages[p.sum_seq0];
+    p.sum_page[0] = p.sum_seq0 < (int)c->summary_pages.size() ? c->summary_pages[p.sum_seq0] : -1;
     p.sum_page[1] = (p.sum_seq0 + 1 < (int)c->summary_pages.size()) ? c->summary_pages[p.sum_seq0 + 1] : -1;
     p.new_sum_seq = -1;
     for (int s = 0; s < S; ++s)
@@ -527,7 +537,7 @@ int gca_get_layout(const gca_cache_t* c, int32_t F, gca_page_entry_t* out, int32
 
 int gca_token_slot(const gca_cache_t* c, int32_t frame, int32_t tau, int32_t* page_id_out, int32_t* slot_out) {
     if (!c || !page_id_out || !slot_out) return GCA_ERR_INVALID_ARG;
-    const int S = c->cfg.summary_tokens;
+    const int S = c->keep;
     if (frame < 0 || frame >= c->T || tau < 0 || tau >= c->Lq) return GCA_ERR_INVALID_ARG;
     if (tau < S) {
         const long long idx = (long long)S * frame + tau;
@@ -549,8 +559,8 @@ int gca_get_info(const gca_cache_t* c, gca_info_t* info) {
     info->image_pages_per_frame = c->ipf;
     info->frames = c->T;
     info->full_frames = (int)c->image_pages.size();
-    info->resident_tokens = (long long)c->cfg.image_tokens * (long long)c->image_pages.size() +
-                            (long long)c->cfg.summary_tokens * c->T;
+    info->resident_tokens = (long long)c->ftok * (long long)c->image_pages.size() +
+                            (long long)c->keep * c->T;
     info->k_pool = c->kpool;
     info->v_pool = c->vpool;
     info->pool_bytes = c->pool_bytes;
