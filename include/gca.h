@@ -244,7 +244,9 @@ const char* gca_status_string(int status);
  * entries gca_get_layout returns), q/out [F][tokens_per_frame][H][64] bf16
  * (device) whose row 0 belongs to frame first_query_frame, lse [F][Lq][H]
  * float32 (device, nullable) and status (device int, nullable: raised like
- * the cache's status word).  Scratch lives in one static device array of
+ * the cache's status word).  summary_tokens is the number of special tokens
+ * each frame keeps in the summary stream (s_k: S, 1 or 0 by the cache's
+ * trajectory_memory).  Scratch lives in one static device array of
  * 18 MiB per GPU: at most 32768 walk entries and 512 partial tiles of 128
  * query rows (ceil(F*Lq/128) * H <= 512), else GCA_ERR_CAPACITY.  The first
  * call on a device looks up the array's address (call it before any stream
