@@ -489,6 +489,20 @@ def run_report(args):
                 cache.evict()
         cache.close()
 
+    # intra-frame attention of one 518x378 frame (the layers that alternate with GCA)
+    w = inputs.METRIC_518x378.with_(L=1)
+    cache = gca.Cache.for_workload(w, max_frames=4)
+    qf, kf, vf = (inputs.draw(w, 3, x, dev)[0] for x in "qkv")
+    outf = torch.empty_like(qf)
+    att = _time_ms(lambda: cache.frame_attention(0, qf, kf, vf, outf))
+    fl = 4.0 * w.Lq * w.Lq * w.H * w.D
+    print(json.dumps({"workload": w.name + " (one frame)", "step": "intra-frame attention",
+                      "Lq": w.Lq, "Lk": w.Lq, "ms_per_layer": att, "tflops": fl / att / 1e9,
+                      "note": "copy of the frame's K/V into transient pages + dense attention; "
+                              "4.1 GFLOP per layer: two launches of a few microseconds each"}),
+          flush=True)
+    cache.close()
+
     # trajectory-memory variants on the 518x378 workload (one layer) at T=10000
     for label, mode, n in (("camera token only", gca.GCA_MEMORY_CAMERA, None),
                            ("sliding window (no memory, no anchors)", gca.GCA_MEMORY_NONE, 0)):

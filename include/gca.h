@@ -198,6 +198,18 @@ int gca_attend(gca_cache_t* cache, int32_t layer, const void* q, int32_t num_que
 int gca_attend_transient(gca_cache_t* cache, int32_t layer, const void* q, const void* k,
                          const void* v, void* out, float* lse, void* stream);
 
+/* Intra-frame attention of one frame for one layer (paper digest §3: the
+ * model alternates intra-frame attention with the cross-frame GCA layers;
+ * news article, pipeline figure): every token of the frame attends to every
+ * token of the same frame, bidirectionally, softmax(scale * q.k), fp32
+ * accumulation; no other frame is read.  q, k, v, out: [S+M][H][D] in the
+ * cache dtype, device or host memory; lse (nullable) [S+M][H] float32.  k and
+ * v go through the layer's transient pages like gca_attend_transient (and
+ * overwrite what a transient call left there); the cache's page table and
+ * frames are neither read nor changed.  Errors: INVALID_ARG, DEVICE_CHECK. */
+int gca_frame_attention(gca_cache_t* cache, int32_t layer, const void* q, const void* k,
+                        const void* v, void* out, float* lse, void* stream);
+
 /* Back to the creation state (windowed mode: state is reset at each window
  * start; code walkthrough §3.3).  Page tables become identical to a fresh
  * cache's; pool bytes are left as they are and never read before rewritten. */

@@ -372,6 +372,37 @@ def test_transient_before_any_keyframe_and_host_pointers(w):
 
 
 # ----------------------------------------------------------------------------
+# intra-frame attention (the layers that alternate with GCA)
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16, inputs.METRIC_518x378.with_(L=2)],
+                         ids=["f32", "bf16", "518x378"])
+def test_frame_attention_is_dense_attention_within_the_frame(w):
+    """Every token attends to the frame's own tokens only; the cache's state is
+    neither read nor changed (it holds other frames here)."""
+    cache = gca.Cache.for_workload(w, max_frames=8)
+    sim = _sim(w, max_frames=8)
+    for t in range(3):
+        cache.append(inputs.draw(w, t, "k", "cuda"), inputs.draw(w, t, "v", "cuda"))
+        sim.append()
+        cache.evict()
+        sim.evict()
+    mirror = Mirror(w, [0])
+    rows = None if w.Lq <= 64 else _rows_sample(w.Lq, extra=8, seed=9)
+    for l in range(w.L):
+        q, k, v = (inputs.draw(w, 100 + l, x, "cuda", layers=[l])[0] for x in "qkv")
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device="cuda")
+        cache.frame_attention(l, q, k, v, out, lse)
+        want, wlse = oracle_transient(mirror, l, q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                      v.float().cpu().numpy(), -1, rows=rows)
+        torch.cuda.synchronize()
+        got, gl = (out, lse) if rows is None else (out[rows], lse[rows])
+        assert max_err(got, want) <= TOL[w.dtype], l
+        assert max_err(gl, wlse) <= LSE_TOL[w.dtype], l
+    assert cache.layout() == sim.walk() and cache.info().frames == 3 and cache.status() == 0
+
+
+# ----------------------------------------------------------------------------
 # the larger workloads
 # ----------------------------------------------------------------------------
 def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, reset=False,

@@ -85,6 +85,7 @@ struct gca_cache {
     int up_F = -1;
     int up_n = 0;
     WalkEntry* d_walk_t = nullptr;   // walk list of the transient (non-keyframe) attention
+    WalkEntry* d_walk_f = nullptr;   // the transient pages alone (frame attention)
     unsigned long long tup_version = 0;
     int tup_n = 0;
     float* ws_o = nullptr;
@@ -112,6 +113,7 @@ void release(gca_cache* c) {
     cudaFree(c->vpool);
     cudaFree(c->d_walk);
     cudaFree(c->d_walk_t);
+    cudaFree(c->d_walk_f);
     cudaFree(c->ws_o);
     cudaFree(c->ws_lse);
     cudaFree(c->st_k);
@@ -285,6 +287,47 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     return GCA_OK;
 }
 
+// A frame's K and V into this layer's transient pages: token u of the frame
+// (summary tokens first) at page u / P, slot u % P.
+int stage_transient(gca_cache* c, int layer, const void* k, const void* v, int frame, cudaStream_t st) {
+    const gca_config_t& g = c->cfg;
+    gca::AppendParams p{};
+    const size_t bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
+    p.k = k;
+    p.v = v;
+    if (!is_device_ptr(k)) {
+        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        p.k = c->st_k;
+    }
+    if (!is_device_ptr(v)) {
+        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
+        p.v = c->st_v;
+    }
+    p.kpool = c->kpool;
+    p.vpool = c->vpool;
+    p.layer0 = layer;
+    p.nlayers = 1;
+    p.Lq = c->Lq;
+    p.S = 0;                 // every token of the frame is laid out like an image token
+    p.M = c->Lq;
+    p.H = g.num_heads;
+    p.P = c->P;
+    p.num_pages = c->num_pages;
+    p.elem_bytes = (int)c->elem;
+    p.sms = c->sms;
+    p.frame = frame;
+    p.sum_seq0 = 0;
+    p.sum_page[0] = p.sum_page[1] = -1;
+    p.new_sum_seq = -1;
+    for (int s = 0; s < c->tpf; ++s) p.img_pages[s] = c->num_regular + s;
+    if (gca::launch_append(p, st) != cudaSuccess) {
+        cudaGetLastError();
+        return GCA_ERR_CUDA;
+    }
+    c->launches += 1;
+    return GCA_OK;
+}
+
 int check_status(const gca_cache* c) {
     return (*(volatile int*)c->h_status) ? GCA_ERR_DEVICE_CHECK : GCA_OK;
 }
@@ -355,7 +398,16 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
               cudaMalloc(&c->vpool, c->pool_bytes) == cudaSuccess;
     c->walk_cap = c->num_pages;
     ok = ok && cudaMalloc(&c->d_walk, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
-         cudaMalloc(&c->d_walk_t, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess;
+         cudaMalloc(&c->d_walk_t, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
+         cudaMalloc(&c->d_walk_f, sizeof(WalkEntry) * c->tpf) == cudaSuccess;
+    if (ok) {
+        // frame attention reads the transient pages only, as frame 0
+        std::vector<WalkEntry> wf(c->tpf);
+        for (int s = 0; s < c->tpf; ++s)
+            wf[s] = make_int4(c->num_regular + s, std::min(c->P, c->Lq - s * c->P), s * c->P, 0);
+        ok = cudaMemcpy(c->d_walk_f, wf.data(), sizeof(WalkEntry) * c->tpf, cudaMemcpyHostToDevice) ==
+             cudaSuccess;
+    }
     for (int i = 0; ok && i < kRing; ++i) {
         ok = cudaHostAlloc((void**)&c->h_stage[i], sizeof(WalkEntry) * c->walk_cap, cudaHostAllocDefault) == cudaSuccess &&
              cudaEventCreateWithFlags(&c->stage_ev[i], cudaEventDisableTiming) == cudaSuccess;
@@ -611,6 +663,17 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
     return run_attention(c, layer, q, F, c->T - F, c->d_walk, c->up_n, out, lse, st);
 }
 
+int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
+                        void* out, float* lse, void* stream) {
+    if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
+    if (layer < 0 || layer >= c->cfg.num_layers) return GCA_ERR_INVALID_ARG;
+    if (int s = check_status(c)) return s;
+    DeviceGuard guard(c->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (int e = stage_transient(c, layer, k, v, 0, st)) return e;
+    return run_attention(c, layer, q, 1, 0, c->d_walk_f, c->tpf, out, lse, st);
+}
+
 int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
                          void* out, float* lse, void* stream) {
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
@@ -638,42 +701,7 @@ int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const voi
         c->tup_n = (int)w.size();
     }
 
-    // the frame's K and V into this layer's transient pages: token u of the
-    // frame (summary tokens first) at page u / P, slot u % P
-    gca::AppendParams p{};
-    const size_t bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
-    p.k = k;
-    p.v = v;
-    if (!is_device_ptr(k)) {
-        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        p.k = c->st_k;
-    }
-    if (!is_device_ptr(v)) {
-        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        p.v = c->st_v;
-    }
-    p.kpool = c->kpool;
-    p.vpool = c->vpool;
-    p.layer0 = layer;
-    p.nlayers = 1;
-    p.Lq = c->Lq;
-    p.S = 0;                 // every token of the frame is laid out like an image token
-    p.M = c->Lq;
-    p.H = g.num_heads;
-    p.P = c->P;
-    p.num_pages = c->num_pages;
-    p.elem_bytes = (int)c->elem;
-    p.sms = c->sms;
-    p.frame = i;
-    p.sum_seq0 = 0;
-    p.sum_page[0] = p.sum_page[1] = -1;
-    p.new_sum_seq = -1;
-    for (int s = 0; s < c->tpf; ++s) p.img_pages[s] = c->num_regular + s;
-    if (gca::launch_append(p, st) != cudaSuccess) {
-        cudaGetLastError();
-        return GCA_ERR_CUDA;
-    }
-    c->launches += 1;
+    if (int e = stage_transient(c, layer, k, v, i, st)) return e;
     return run_attention(c, layer, q, 1, i, c->d_walk_t, c->tup_n, out, lse, st);
 }
 }  // extern "C"

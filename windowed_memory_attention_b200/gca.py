@@ -26,7 +26,7 @@ STATUS = {0: "GCA_OK", 1: "GCA_ERR_INVALID_ARG", 2: "GCA_ERR_CAPACITY", 3: "GCA_
 EXPORTS = ("gca_cache_create", "gca_cache_destroy", "gca_append_frame", "gca_evict_to_summary",
            "gca_attend", "gca_reset", "gca_get_layout", "gca_token_slot", "gca_get_info",
            "gca_device_status", "gca_status_string", "gca_attend_pages_noalloc",
-           "gca_selftest_bounded_wait", "gca_attend_transient")
+           "gca_selftest_bounded_wait", "gca_attend_transient", "gca_frame_attention")
 
 
 class gca_config_t(ctypes.Structure):
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "gca_evict_to_summary": [vp, ctypes.POINTER(i32)],
             "gca_attend": [vp, i32, vp, i32, vp, vp, vp],
             "gca_attend_transient": [vp, i32, vp, vp, vp, vp, vp, vp],
+            "gca_frame_attention": [vp, i32, vp, vp, vp, vp, vp, vp],
             "gca_reset": [vp],
             "gca_get_layout": [vp, i32, ctypes.POINTER(gca_page_entry_t), i32, ctypes.POINTER(i32)],
             "gca_token_slot": [vp, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
@@ -163,6 +164,12 @@ def gca_attend_transient(cache, layer: int, q: torch.Tensor, k: torch.Tensor, v:
                                                               _ptr(out), _ptr(lse), _stream(stream)))
 
 
+def gca_frame_attention(cache, layer: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        out: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check("gca_frame_attention", lib().gca_frame_attention(cache, layer, _ptr(q), _ptr(k), _ptr(v),
+                                                            _ptr(out), _ptr(lse), _stream(stream)))
+
+
 def gca_reset(cache) -> None:
     _check("gca_reset", lib().gca_reset(cache))
 
@@ -243,6 +250,9 @@ class Cache:
 
     def attend_transient(self, layer, q, k, v, out, lse=None, stream=None):
         gca_attend_transient(self.handle, layer, q, k, v, out, lse, stream)
+
+    def frame_attention(self, layer, q, k, v, out, lse=None, stream=None):
+        gca_frame_attention(self.handle, layer, q, k, v, out, lse, stream)
 
     def reset(self):
         gca_reset(self.handle)
