@@ -28,6 +28,15 @@ __device__ __forceinline__ int4 ld_stream(const int4* p) {
     return r;
 }
 
+#ifndef GCA_APPEND_U
+#define GCA_APPEND_U 4
+#endif
+#ifndef GCA_APPEND_BLOCKS_PER_SM
+#define GCA_APPEND_BLOCKS_PER_SM 8
+#endif
+
+// HSHIFT = log2(H) when H is a power of two (shifts instead of divisions), else -1
+template <int HSHIFT>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     const int lt = blockIdx.y;                 // layer-local index * 2 + tensor
     const int ll = lt >> 1;
@@ -48,6 +57,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     const unsigned H = (unsigned)p.H;
     const unsigned n_copy = (unsigned)p.Lq * H * cpr;
     // zero regions, per head: image tail slots and new summary page tail
+    const int p_shift = p.P == 128 ? 7 : 6;              // P is 64 or 128
     const unsigned img_tail = (p.M % p.P) ? (unsigned)(p.P - p.M % p.P) : 0u;
     unsigned sum_from = 0, sum_tail = 0;
     if (p.new_sum_seq >= 0) {
@@ -64,19 +74,18 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
             zero = false;
             const unsigned chunk = u & (cpr - 1);
             const unsigned th = u >> cpr_shift;
-            const unsigned tau = th / H;
-            const unsigned h = th - tau * H;
+            const unsigned tau = HSHIFT >= 0 ? th >> HSHIFT : th / H;
+            const unsigned h = HSHIFT >= 0 ? th & ((1u << (HSHIFT & 31)) - 1u) : th - tau * H;
             int page, slot;
             if ((int)tau < p.S) {
                 const int idx = p.S * p.frame + (int)tau;
-                const int seq = idx / p.P;
+                const int seq = idx >> p_shift;
                 page = p.sum_page[seq - p.sum_seq0];
-                slot = idx - seq * p.P;
+                slot = idx & (p.P - 1);
             } else {
                 const int m = (int)tau - p.S;
-                const int seq = m / p.P;
-                page = p.img_pages[seq];
-                slot = m - seq * p.P;
+                page = p.img_pages[m >> p_shift];
+                slot = m & (p.P - 1);
             }
             return lpool + ((long long)page * p.H + h) * tile_bytes +
                    (long long)slot * row_bytes + chunk * 16;
@@ -104,7 +113,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     };
 
     // four independent chunks per thread per iteration: loads first, then stores
-    constexpr int U = 4;
+    constexpr int U = GCA_APPEND_U;
     const unsigned stride = gridDim.x * blockDim.x;
     for (unsigned base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += U * stride) {
         int4 val[U];
@@ -131,13 +140,23 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     const int sms = p.sms > 0 ? p.sms : 148;
     const long long per_lt = (long long)p.Lq * p.H * (kHeadDim * p.elem_bytes / 16);
-    // about 4 chunks per thread per (layer, tensor), at most 8 blocks per SM overall
-    long long want = (per_lt + 256 * 4 - 1) / (256 * 4);
-    const long long cap = (8LL * sms + 2 * p.nlayers - 1) / (2 * p.nlayers);
+    // about U chunks per thread per (layer, tensor), a bounded number of blocks per SM overall
+    constexpr int U = GCA_APPEND_U;
+    long long want = (per_lt + 256 * U - 1) / (256 * U);
+    const long long cap = ((long long)GCA_APPEND_BLOCKS_PER_SM * sms + 2 * p.nlayers - 1) / (2 * p.nlayers);
     if (want > cap) want = cap;
     if (want < 1) want = 1;
     dim3 grid((unsigned)want, (unsigned)(2 * p.nlayers));
-    append_kernel<<<grid, 256, 0, s>>>(p);
+    const int hs = (p.H & (p.H - 1)) == 0 ? __builtin_ctz((unsigned)p.H) : -1;
+    switch (hs) {
+        case 0: append_kernel<0><<<grid, 256, 0, s>>>(p); break;
+        case 1: append_kernel<1><<<grid, 256, 0, s>>>(p); break;
+        case 2: append_kernel<2><<<grid, 256, 0, s>>>(p); break;
+        case 3: append_kernel<3><<<grid, 256, 0, s>>>(p); break;
+        case 4: append_kernel<4><<<grid, 256, 0, s>>>(p); break;
+        case 5: append_kernel<5><<<grid, 256, 0, s>>>(p); break;
+        default: append_kernel<-1><<<grid, 256, 0, s>>>(p); break;
+    }
     return cudaGetLastError();
 }
 
