@@ -58,6 +58,10 @@ def parse():
                     help="instead of the bench line: per-layer attention / append timings of "
                          "the worked-example stream at T=100/1000/10000, the dense causal "
                          "limit at T=1000 and one windowed-VO window, one JSON line each")
+    ap.add_argument("--append-probe", type=int, default=0, metavar="FRAMES",
+                    help="instead of the bench line: FRAMES appends of the 518x378 workload's 24 "
+                         "layers into a small cache (window 4, about 1 GB of pools) with the append "
+                         "timed; a small command for profiler captures of the append kernel")
     return ap.parse_args()
 
 
@@ -443,6 +447,37 @@ def _time_ms(fn, reps=20, warm=3):
     return e0.elapsed_time(e1) / reps
 
 
+def run_append_probe(args):
+    """Append launches of the full 24-layer frame into a cache with a short window:
+    the append's work per launch does not depend on the window, the pools do."""
+    pk = peaks()
+    dev = torch.device("cuda", 0)
+    w = inputs.METRIC_518x378.with_(k=4)
+    cache = gca.Cache.for_workload(w, max_frames=args.append_probe + 1)
+    kv = [(inputs.draw(w, t, "k", dev), inputs.draw(w, t, "v", dev)) for t in range(4)]
+    # back-to-back launches between two events: the host runs ahead of the GPU,
+    # so the per-launch figure is the kernels' own time plus the launch gaps
+    half = args.append_probe // 2
+    for t in range(half):
+        cache.append(*kv[t % 4])
+        cache.evict()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(half, args.append_probe):
+        cache.append(*kv[t % 4])
+        cache.evict()
+    e1.record()
+    torch.cuda.synchronize()
+    if cache.status() != 0:
+        raise RuntimeError("device status word raised")
+    med = e0.elapsed_time(e1) / (args.append_probe - half)
+    b = 2 * 2 * w.L * w.Lq * w.H * w.D * 2
+    print(json.dumps({"append_probe": w.name + " (window 4)", "frames": args.append_probe,
+                      "us_per_launch": med * 1e3, "bytes_per_launch": b, "GBs": b / (med / 1e3) / 1e9,
+                      "frac_hbm": b / (med / 1e3) / 1e9 / pk["hbm"]}), flush=True)
+
+
 def run_report(args):
     """Attention and append timings per layer on the other workloads."""
     pk = peaks()
@@ -554,6 +589,9 @@ def main():
     torch.cuda.set_device(local_rank)
     if args.report:
         run_report(args)
+        return
+    if args.append_probe:
+        run_append_probe(args)
         return
     if world > 1:
         import datetime
