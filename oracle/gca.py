@@ -27,7 +27,7 @@ Sources (LingBot-Map pages):
     K/V is not kept (skip-append); §3.3: the window counts keyframes entering
     the cache, not video frames.
 
-Readings where the pages leave a step open (each is listed in the design doc):
+Readings where the pages leave a step open:
   * the k-frame window counts the current frame, so after frame t the full
     frames are the anchors and t-k+1..t — the only reading under which the
     cache holds exactly M(n+k)+6T tokens once T > n+k;
