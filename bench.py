@@ -58,6 +58,10 @@ def parse():
                     help="instead of the bench line: per-layer attention / append timings of "
                          "the worked-example stream at T=100/1000/10000, the dense causal "
                          "limit at T=1000 and one windowed-VO window, one JSON line each")
+    ap.add_argument("--report-oracle", action="store_true",
+                    help="instead of the bench line: the CPU oracle's time per layer-step at the "
+                         "report points (worked example and 518x378 at T=100/1000/10000, dense "
+                         "limit at T=1000) on the host cores; no GPU work")
     ap.add_argument("--append-probe", type=int, default=0, metavar="FRAMES",
                     help="instead of the bench line: FRAMES appends of the 518x378 workload's 24 "
                          "layers into a small cache (window 4, about 1 GB of pools) with the append "
@@ -478,6 +482,37 @@ def run_append_probe(args):
                       "frac_hbm": b / (med / 1e3) / 1e9 / pk["hbm"]}), flush=True)
 
 
+def run_oracle_report(args):
+    """cpu_baseline of the report points: the oracle's attention core as it stands, on a bounded
+    sample (64 query rows of one head) of each point's shape, scaled to all rows and heads.  The
+    inputs are seeded random arrays of the point's shape: the core's time does not depend on the
+    values.  The key gather of the bench line's cpu_baseline is not included."""
+    from oracle import gca as ogca
+    import numpy as np
+    points = [(inputs.WORKED_EXAMPLE, T) for T in (100, 1000, 10000)] + \
+             [(inputs.METRIC_518x378, T) for T in (100, 1000, 10000)] + [(inputs.DENSE_CAUSAL, 1000)]
+    rows, heads = 64, 1
+    cores = ogca.core_threads()
+    rng = np.random.default_rng(0)
+    for w, T in points:
+        lk = lk_at(w, T)
+        q = rng.standard_normal((rows, heads, w.D), dtype=np.float32)
+        k = rng.standard_normal((lk, heads, w.D), dtype=np.float32)
+        v = rng.standard_normal((lk, heads, w.D), dtype=np.float32)
+        ogca.attention_c(q[:4], k, v, w.softmax_scale)          # warm the core once
+        t0 = time.perf_counter()
+        ogca.attention_c(q, k, v, w.softmax_scale)
+        dt = time.perf_counter() - t0
+        step_s = dt * (w.Lq / rows) * (w.H / heads)
+        print(json.dumps({"workload": w.name, "T": T, "Lq": w.Lq, "Lk": lk,
+                          "cpu_baseline": {"value": 1.0 / step_s, "unit": UNIT, "cores": cores,
+                                           "kind": "oracle", "ms_per_layer": step_s * 1e3,
+                                           "sample": f"{rows} query rows x {heads} head against all "
+                                                     f"{lk} keys, seeded random inputs of the point's "
+                                                     f"shape, scaled to {w.Lq} rows x {w.H} heads; "
+                                                     f"key gather not included"}}), flush=True)
+
+
 def run_report(args):
     """Attention and append timings per layer on the other workloads."""
     pk = peaks()
@@ -585,6 +620,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args)
+        return
+    if args.report_oracle:
+        run_oracle_report(args)
         return
     torch.cuda.set_device(local_rank)
     if args.report:
