@@ -52,6 +52,7 @@ extern "C" {
 #endif
 
 #define GCA_ALL_LAYERS (-1)
+#define GCA_HOST_ONLY (-1)   /* gca_cache_create device: the page table alone */
 
 typedef enum {
     GCA_OK = 0,
@@ -135,9 +136,14 @@ typedef struct {
  *           + ceil(s_k * max_frames / P) pages the allocator hands out,
  *           + ceil((S+M) / P)            transient pages after them
  *                                        (gca_attend_transient), per layer.
- * Errors: INVALID_ARG (non-positive sizes, null out), UNSUPPORTED (head_dim
- * != 64, page_size not 64/128, unknown dtype, ceil((S+M)/P) > 128), CUDA
- * (allocation). */
+ * device = GCA_HOST_ONLY creates the page table alone, with no device state:
+ * gca_append_frame (k and v may be NULL; nothing is copied), evict, reset,
+ * get_layout, token_slot, get_info and device_status behave as on a device;
+ * the attention calls and the self-test return UNSUPPORTED.  It lets a host
+ * without a GPU check the page table.
+ * Errors: INVALID_ARG (non-positive sizes, null out, no such device),
+ * UNSUPPORTED (head_dim != 64, page_size not 64/128, unknown dtype,
+ * ceil((S+M)/P) > 128), CUDA (allocation). */
 int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out);
 
 /* Free everything the cache owns.  The caller must have synchronised the

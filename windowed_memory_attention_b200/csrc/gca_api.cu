@@ -100,12 +100,18 @@ struct gca_cache {
     void* st_out = nullptr;
     float* st_lse = nullptr;
     long long launches = 0;
+    bool host_only = false;   // GCA_HOST_ONLY: the page table alone, no device state
 };
 
 namespace {
 
 void release(gca_cache* c) {
     if (!c) return;
+    if (c->host_only) {
+        delete c->h_status;
+        delete c;
+        return;
+    }
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(c->device);
@@ -133,11 +139,14 @@ void release(gca_cache* c) {
 // Restores the caller's current device on scope exit.
 struct DeviceGuard {
     int prev = -1;
-    explicit DeviceGuard(int dev) {
+    bool active = false;      // a host-only cache (device < 0) touches no device
+    explicit DeviceGuard(int dev) : active(dev >= 0) {
+        if (!active) return;
         cudaGetDevice(&prev);
         if (prev != dev) cudaSetDevice(dev);
     }
     ~DeviceGuard() {
+        if (!active) return;
         int now = -1;
         cudaGetDevice(&now);
         if (prev >= 0 && now != prev) cudaSetDevice(prev);
@@ -364,8 +373,9 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     // a frame's image pages, and a non-keyframe's transient pages, fit one append launch
     if ((g.image_tokens + g.summary_tokens + g.page_size - 1) / g.page_size > gca::kMaxImagePages)
         return GCA_ERR_UNSUPPORTED;
+    const bool host = device == GCA_HOST_ONLY;
     int ndev = 0;
-    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    if (!host && (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)) {
         cudaGetLastError();
         return GCA_ERR_INVALID_ARG;
     }
@@ -374,7 +384,8 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     gca_cache* c = new gca_cache();
     c->cfg = g;
     c->device = device;
-    cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, device);
+    c->host_only = host;
+    if (!host) cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, device);
     c->P = g.page_size;
     c->keep = g.trajectory_memory == GCA_MEMORY_SUMMARY ? g.summary_tokens
             : g.trajectory_memory == GCA_MEMORY_CAMERA ? 1 : 0;
@@ -394,9 +405,14 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
 
     const size_t tile = (size_t)c->P * gca::kHeadDim * c->elem;
     c->pool_bytes = (size_t)g.num_layers * c->num_pages * g.num_heads * tile;
+    c->walk_cap = c->num_pages;
+    if (host) {
+        c->h_status = new int(0);
+        *out = c;
+        return GCA_OK;
+    }
     bool ok = cudaMalloc(&c->kpool, c->pool_bytes) == cudaSuccess &&
               cudaMalloc(&c->vpool, c->pool_bytes) == cudaSuccess;
-    c->walk_cap = c->num_pages;
     ok = ok && cudaMalloc(&c->d_walk, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
          cudaMalloc(&c->d_walk_t, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
          cudaMalloc(&c->d_walk_f, sizeof(WalkEntry) * c->tpf) == cudaSuccess;
@@ -459,7 +475,7 @@ int gca_cache_destroy(gca_cache_t* c) {
 
 int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v,
                      int64_t* frame_index_out, void* stream) {
-    if (!c || !k || !v) return GCA_ERR_INVALID_ARG;
+    if (!c || (!c->host_only && (!k || !v))) return GCA_ERR_INVALID_ARG;
     const gca_config_t& g = c->cfg;
     if (layer != GCA_ALL_LAYERS && (layer < 0 || layer >= g.num_layers)) return GCA_ERR_INVALID_ARG;
     if (int s = check_status(c)) return s;
@@ -498,6 +514,11 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
         t = c->T - 1;
         l0 = layer;
         nl = 1;
+    }
+    if (c->host_only) {       // page table only: nothing to copy
+        for (int l = l0; l < l0 + nl; ++l) c->layer_frames[l] = t + 1;
+        if (frame_index_out) *frame_index_out = t;
+        return GCA_OK;
     }
 
     gca::AppendParams p{};
@@ -630,6 +651,7 @@ int gca_device_status(gca_cache_t* c, int32_t* status_out, int32_t clear) {
 
 int gca_selftest_bounded_wait(gca_cache_t* c, int32_t timeout_ms, int32_t* status_out) {
     if (!c || !status_out || timeout_ms < 1 || timeout_ms > 10000) return GCA_ERR_INVALID_ARG;
+    if (c->host_only) return GCA_ERR_UNSUPPORTED;
     DeviceGuard guard(c->device);
     if (gca::launch_bounded_wait_selftest(c->d_status, (unsigned long long)timeout_ms * 1000000ull, 0) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
@@ -643,6 +665,7 @@ int gca_selftest_bounded_wait(gca_cache_t* c, int32_t timeout_ms, int32_t* statu
 int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* out, float* lse,
                void* stream) {
     if (!c || !q || !out) return GCA_ERR_INVALID_ARG;
+    if (c->host_only) return GCA_ERR_UNSUPPORTED;
     const gca_config_t& g = c->cfg;
     if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
     if (F < 1 || F > g.max_query_frames) return GCA_ERR_INVALID_ARG;
@@ -666,6 +689,7 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
 int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
                         void* out, float* lse, void* stream) {
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
+    if (c->host_only) return GCA_ERR_UNSUPPORTED;
     if (layer < 0 || layer >= c->cfg.num_layers) return GCA_ERR_INVALID_ARG;
     if (int s = check_status(c)) return s;
     DeviceGuard guard(c->device);
@@ -677,6 +701,7 @@ int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void
 int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
                          void* out, float* lse, void* stream) {
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
+    if (c->host_only) return GCA_ERR_UNSUPPORTED;
     const gca_config_t& g = c->cfg;
     if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
     if (c->layer_frames[layer] != c->T) return GCA_ERR_STATE;

@@ -18,6 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgca.so")
 
 GCA_ALL_LAYERS = -1
+GCA_HOST_ONLY = -1        # cache-create device: the page table alone (no GPU needed)
 GCA_DTYPE_BF16, GCA_DTYPE_F32 = 0, 1
 GCA_PAGE_IMAGE, GCA_PAGE_SUMMARY = 0, 1
 GCA_MEMORY_SUMMARY, GCA_MEMORY_CAMERA, GCA_MEMORY_NONE = 0, 1, 2
