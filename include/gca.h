@@ -228,11 +228,21 @@ int gca_reset(gca_cache_t* cache);
 int gca_get_layout(const gca_cache_t* cache, int32_t num_query_frames,
                    gca_page_entry_t* out, int32_t cap, int32_t* n_out);
 
-/* (page id, slot) of token slot tau of frame `frame` (tau < S: summary).
- * Errors: INVALID_ARG (frame not appended, tau out of range), STATE (the
- * frame's image tokens were evicted and tau >= S). */
+/* (page id, slot) of token slot tau of frame `frame` (tau < s_k: summary
+ * stream, else the frame's image pages).  Errors: INVALID_ARG (frame not
+ * appended, tau out of range), STATE (the frame's image pages were evicted
+ * and tau >= s_k). */
 int gca_token_slot(const gca_cache_t* cache, int32_t frame, int32_t tau,
                    int32_t* page_id_out, int32_t* slot_out);
+
+/* The per-frame mask the attention kernels apply (paper digest §2.5, with the
+ * cache's n, k, s_k and anchor_block): how many tokens of walk-list entry
+ * *entry query frame `query_frame` may see.  The visible tokens of a page are
+ * always its first *prefix_out slots, so one integer per (frame, page) is the
+ * whole mask.  For tests and tools; works on host-only caches.
+ * Errors: INVALID_ARG (null pointer, negative query frame). */
+int gca_visible_prefix(const gca_cache_t* cache, const gca_page_entry_t* entry,
+                       int32_t query_frame, int32_t* prefix_out);
 
 int gca_get_info(const gca_cache_t* cache, gca_info_t* info);
 

@@ -626,6 +626,15 @@ int gca_token_slot(const gca_cache_t* c, int32_t frame, int32_t tau, int32_t* pa
     return GCA_OK;
 }
 
+int gca_visible_prefix(const gca_cache_t* c, const gca_page_entry_t* e, int32_t query_frame,
+                       int32_t* prefix_out) {
+    if (!c || !e || !prefix_out || query_frame < 0) return GCA_ERR_INVALID_ARG;
+    const gca::MaskRule rule{c->cfg.num_anchor, c->cfg.window, c->keep, c->cfg.anchor_block ? 1 : 0};
+    const int4 w = make_int4(e->page_id, e->n_valid, e->first, e->kind == GCA_PAGE_IMAGE ? e->frame : -1);
+    *prefix_out = gca::visible_prefix(rule, w, query_frame);
+    return GCA_OK;
+}
+
 int gca_get_info(const gca_cache_t* c, gca_info_t* info) {
     if (!c || !info) return GCA_ERR_INVALID_ARG;
     info->num_pages = c->num_pages;

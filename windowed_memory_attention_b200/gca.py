@@ -27,7 +27,8 @@ STATUS = {0: "GCA_OK", 1: "GCA_ERR_INVALID_ARG", 2: "GCA_ERR_CAPACITY", 3: "GCA_
 EXPORTS = ("gca_cache_create", "gca_cache_destroy", "gca_append_frame", "gca_evict_to_summary",
            "gca_attend", "gca_reset", "gca_get_layout", "gca_token_slot", "gca_get_info",
            "gca_device_status", "gca_status_string", "gca_attend_pages_noalloc",
-           "gca_selftest_bounded_wait", "gca_attend_transient", "gca_frame_attention")
+           "gca_selftest_bounded_wait", "gca_attend_transient", "gca_frame_attention",
+           "gca_visible_prefix")
 
 
 class gca_config_t(ctypes.Structure):
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "gca_attend": [vp, i32, vp, i32, vp, vp, vp],
             "gca_attend_transient": [vp, i32, vp, vp, vp, vp, vp, vp],
             "gca_frame_attention": [vp, i32, vp, vp, vp, vp, vp, vp],
+            "gca_visible_prefix": [vp, ctypes.POINTER(gca_page_entry_t), i32, ctypes.POINTER(i32)],
             "gca_reset": [vp],
             "gca_get_layout": [vp, i32, ctypes.POINTER(gca_page_entry_t), i32, ctypes.POINTER(i32)],
             "gca_token_slot": [vp, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
@@ -191,6 +193,15 @@ def gca_token_slot(cache, frame: int, tau: int) -> Tuple[int, int]:
     return pid.value, slot.value
 
 
+def gca_visible_prefix(cache, entry, query_frame: int) -> int:
+    """Visible-prefix length of a walk-list entry (page_id, kind, frame, first, n_valid)."""
+    e = gca_page_entry_t(*entry)
+    n = ctypes.c_int32(0)
+    _check("gca_visible_prefix", lib().gca_visible_prefix(cache, ctypes.byref(e), query_frame,
+                                                          ctypes.byref(n)))
+    return n.value
+
+
 def gca_get_info(cache) -> gca_info_t:
     info = gca_info_t()
     _check("gca_get_info", lib().gca_get_info(cache, ctypes.byref(info)))
@@ -263,6 +274,9 @@ class Cache:
 
     def info(self) -> gca_info_t:
         return gca_get_info(self.handle)
+
+    def visible_prefix(self, entry, query_frame: int) -> int:
+        return gca_visible_prefix(self.handle, entry, query_frame)
 
     def token_slot(self, frame: int, tau: int):
         return gca_token_slot(self.handle, frame, tau)
