@@ -31,6 +31,8 @@
 #include <set>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/gca.h"
 #include "gca_internal.h"
 
@@ -135,6 +137,12 @@ void release(gca_cache* c) {
     cudaSetDevice(prev);
     delete c;
 }
+
+// An NVTX range around one public call (a no-op unless a profiler attached one).
+struct Range {
+    explicit Range(const char* name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+};
 
 // Restores the caller's current device on scope exit.
 struct DeviceGuard {
@@ -475,6 +483,7 @@ int gca_cache_destroy(gca_cache_t* c) {
 
 int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v,
                      int64_t* frame_index_out, void* stream) {
+    Range range("gca_append_frame");
     if (!c || (!c->host_only && (!k || !v))) return GCA_ERR_INVALID_ARG;
     const gca_config_t& g = c->cfg;
     if (layer != GCA_ALL_LAYERS && (layer < 0 || layer >= g.num_layers)) return GCA_ERR_INVALID_ARG;
@@ -566,6 +575,7 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
 }
 
 int gca_evict_to_summary(gca_cache_t* c, int32_t* frames_evicted_out) {
+    Range range("gca_evict_to_summary");
     if (!c) return GCA_ERR_INVALID_ARG;
     const int t = c->T - 1;
     int count = 0;
@@ -585,6 +595,7 @@ int gca_evict_to_summary(gca_cache_t* c, int32_t* frames_evicted_out) {
 }
 
 int gca_reset(gca_cache_t* c) {
+    Range range("gca_reset");
     if (!c) return GCA_ERR_INVALID_ARG;
     c->free_pages.clear();
     for (int i = 0; i < c->num_regular; ++i) c->free_pages.insert(i);
@@ -673,6 +684,7 @@ int gca_selftest_bounded_wait(gca_cache_t* c, int32_t timeout_ms, int32_t* statu
 
 int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* out, float* lse,
                void* stream) {
+    Range range("gca_attend");
     if (!c || !q || !out) return GCA_ERR_INVALID_ARG;
     if (c->host_only) return GCA_ERR_UNSUPPORTED;
     const gca_config_t& g = c->cfg;
@@ -697,6 +709,7 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
 
 int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
                         void* out, float* lse, void* stream) {
+    Range range("gca_frame_attention");
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
     if (c->host_only) return GCA_ERR_UNSUPPORTED;
     if (layer < 0 || layer >= c->cfg.num_layers) return GCA_ERR_INVALID_ARG;
@@ -709,6 +722,7 @@ int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void
 
 int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
                          void* out, float* lse, void* stream) {
+    Range range("gca_attend_transient");
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
     if (c->host_only) return GCA_ERR_UNSUPPORTED;
     const gca_config_t& g = c->cfg;
