@@ -167,3 +167,33 @@ def test_attention_is_unsupported_without_a_device():
         assert e.value.name == "GCA_ERR_UNSUPPORTED"
     assert cache.status() == 0
     cache.close()
+
+
+def test_null_and_range_arguments_are_rejected():
+    import ctypes
+    w = inputs.TINY
+    cache, _ = _pair(w)
+    cache.append(None, None)
+    L = gca.lib()
+    n = ctypes.c_int32(0)
+    e = gca.gca_page_entry_t(0, gca.GCA_PAGE_IMAGE, 0, 0, 16)
+    assert gca.STATUS[L.gca_get_layout(cache.handle, 1, None, 0, None)] == "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_get_layout(cache.handle, 1, None, 4, ctypes.byref(n))] == "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_token_slot(cache.handle, 0, 0, None, None)] == "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_visible_prefix(cache.handle, None, 0, ctypes.byref(n))] == "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_visible_prefix(cache.handle, ctypes.byref(e), -1, ctypes.byref(n))] == \
+        "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_get_info(None, None)] == "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_evict_to_summary(None, None)] == "GCA_ERR_INVALID_ARG"
+    assert gca.STATUS[L.gca_reset(None)] == "GCA_ERR_INVALID_ARG"
+    with pytest.raises(gca.GCAError) as err:
+        cache.token_slot(1, 0)                      # frame not appended
+    assert err.value.name == "GCA_ERR_INVALID_ARG"
+    with pytest.raises(gca.GCAError) as err:
+        cache.token_slot(0, w.Lq)                   # tau out of range
+    assert err.value.name == "GCA_ERR_INVALID_ARG"
+    with pytest.raises(gca.GCAError) as err:
+        gca.Cache.for_workload(w, device=gca.GCA_HOST_ONLY, trajectory_memory=3)
+    assert err.value.name == "GCA_ERR_INVALID_ARG"
+    assert L.gca_cache_destroy(None) == 0            # null is accepted
+    cache.close()

@@ -349,6 +349,27 @@ def test_allocator_memory_variants_follow_closed_form(keep):
             assert pid == sim.image_pages[t][(tau - keep) // 128] and slot == (tau - keep) % 128
 
 
+@pytest.mark.parametrize("keep,n", [(1, 2), (0, 0)])
+def test_transient_key_count_with_memory_variants(keep, n):
+    """A non-keyframe over a camera-only or memory-free cache: Q = 0 gives
+    lse = ln(every token of the min(K, n+k) full keyframes + keep tokens of the
+    other K keyframes + the frame's own S+M), K = keyframes cached so far."""
+    M, S, k, X, interval = 5, 6, 3, 15, 2
+    Q, K, V = _rand_stream(X, M, 1, 8, seed=41, S=S)
+    Q[:] = 0
+    keys = [y for y in range(X) if gca.is_keyframe(y, n=n, interval=interval)]
+    fkv = _frame_kv(K[keys], V[keys])
+    for x in range(X):
+        if gca.is_keyframe(x, n=n, interval=interval):
+            continue
+        cached = x + 1 if x < n else n + (x - n) // interval + 1
+        _, lse = gca.transient_step(Q[x], K[x], V[x], cached - 1, fkv, n=n, k=k, S=S,
+                                    scale=0.125, impl="np", keep=keep)
+        full = min(cached, n + k)
+        want = math.log((M + S) * full + keep * (cached - full) + (M + S))
+        assert np.allclose(lse, want, atol=1e-12, rtol=0), x
+
+
 def test_single_frame_is_plain_attention():
     Q, K, V = _rand_stream(1, 11, 2, 16, seed=5)
     scale = 0.25
