@@ -643,3 +643,28 @@ def test_planted_sliding_window_with_anchor_leak_is_caught(monkeypatch):
         return orig(i, j, tau, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
     monkeypatch.setattr(gca, "visible", wrong)
     assert not pin_sliding_window_is_banded_sdpa()
+
+
+def test_planted_camera_only_keeping_the_wrong_token_is_caught(monkeypatch):
+    # keeps one token per old frame, but the anchor token (slot 1) instead of the
+    # camera token (slot 0): the key count is unchanged, the brute force differs
+    orig = gca.gather_keys
+
+    def wrong(i, frame_kv, *, n, k, S, anchor_block=False, keep=None):
+        if keep != 1:
+            return orig(i, frame_kv, n=n, k=k, S=S, anchor_block=anchor_block, keep=keep)
+        shifted = lambda j, summary_only: tuple(a[1:] for a in frame_kv(j, summary_only))
+        full, summary = gca.stream_state(i, n=n, k=k, anchor_block=anchor_block)
+        ks, vs = [], []
+        for f in full:
+            kf, vf = frame_kv(f, False)
+            ks.append(kf)
+            vs.append(vf)
+        for f in summary:
+            kf, vf = shifted(f, True)
+            ks.append(kf[:1])
+            vs.append(vf[:1])
+        return np.concatenate(ks, 0), np.concatenate(vs, 0)
+    monkeypatch.setattr(gca, "gather_keys", wrong)
+    with pytest.raises(AssertionError):
+        test_memory_variants_stream_equals_bruteforce(1, 2, False)
