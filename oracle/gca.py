@@ -362,3 +362,84 @@ def frame_visibility_matrix(T: int, *, n: int, k: int, S: int, anchor_block: boo
             row.append("F" if img and summ else ("S" if summ else "."))
         rows.append("".join(row))
     return rows
+
+
+# ----------------------------------------------------------------------------
+# 3D rotary position encoding (video RoPE) on Q and K
+# ----------------------------------------------------------------------------
+# Sources: the news article's ablation (context tokens together with video RoPE
+# raise AUC@3), paper digest §2.7 (a temporal positional encoding PE(t) on the
+# trajectory memory's summary tokens, taken from the WAN video model), the code
+# walkthrough §3.1 (enable_3d_rope is a first-class constructor flag) and the
+# paper-to-code article §3 (3D RoPE carries the position along the time axis).
+# The formula is not printed; the reading taken here is rotary position
+# encoding (Su et al., "RoFormer", 2021) over three axes, time t, patch row y
+# and patch column x:
+#   * the D=64 head dims are split into three contiguous parts, 24 dims for t,
+#     20 for y, 20 for x (time takes the larger share);
+#   * inside a part of d dims, dims (2i, 2i+1) form pair i, rotated by the angle
+#     pos * base^(-2i/d) with base 10000: (a, b) -> (a cos - b sin, a sin + b cos);
+#   * image token m of frame t (row-major over a grid_w-wide patch grid) sits at
+#     (t, m // grid_w, m % grid_w); the frame's special tokens at (t, 0, 0), so
+#     they carry only the timestamp;
+#   * t is the frame's index in the cache (frames since create or reset);
+#   * Q and K are rotated, V is not; the rotated vectors are held in the
+#     workload's dtype, as a model running in that dtype holds them.
+ROPE_SPLIT = (24, 20, 20)
+ROPE_BASE = 10000.0
+
+
+def rope_angles(t: float, y: float, x: float, D: int = 64, base: float = ROPE_BASE,
+                split=ROPE_SPLIT) -> np.ndarray:
+    """Rotation angle of each of the D/2 dim pairs at position (t, y, x)."""
+    assert sum(split) == D and all(d % 2 == 0 for d in split)
+    out = []
+    for pos, d in zip((t, y, x), split):
+        i = np.arange(d // 2, dtype=np.float64)
+        out.append(pos * base ** (-2.0 * i / d))
+    return np.concatenate(out)
+
+
+def rope_matrix(t: float, y: float, x: float, D: int = 64, base: float = ROPE_BASE,
+                split=ROPE_SPLIT) -> np.ndarray:
+    """The explicit [D][D] rotation: block diagonal, one 2x2 rotation per pair."""
+    R = np.zeros((D, D), dtype=np.float64)
+    for i, a in enumerate(rope_angles(t, y, x, D, base, split)):
+        c, s = math.cos(a), math.sin(a)
+        R[2 * i, 2 * i], R[2 * i, 2 * i + 1] = c, -s
+        R[2 * i + 1, 2 * i], R[2 * i + 1, 2 * i + 1] = s, c
+    return R
+
+
+def token_positions(frame: int, S: int, M: int, grid_w: int):
+    """(t, y, x) of the S + M tokens of a frame (special tokens first)."""
+    pos = [(frame, 0, 0)] * S
+    pos += [(frame, m // grid_w, m % grid_w) for m in range(M)]
+    return pos
+
+
+def round_to_dtype(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Values as held in `dtype` ("f32" or "bf16", round to nearest even),
+    returned as float64.  bf16 keeps the top 16 bits of the float32 pattern."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    if dtype == "f32":
+        return f.astype(np.float64)
+    b = f.view(np.uint32).astype(np.uint64)
+    b = (b + np.uint64(0x7FFF) + ((b >> np.uint64(16)) & np.uint64(1))) & np.uint64(0xFFFF0000)
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def rope_frame(x: np.ndarray, frame: int, *, S: int, grid_w: int, dtype: str,
+               base: float = ROPE_BASE) -> np.ndarray:
+    """Rotate every token of one frame, x [S+M][H][D], by its position's
+    explicit rotation matrix (the same for every head), then hold the result
+    in `dtype`.  Returns float32."""
+    Lq, H, D = x.shape
+    out = np.empty((Lq, H, D), dtype=np.float64)
+    cache = {}
+    for u, p in enumerate(token_positions(frame, S, Lq - S, grid_w)):
+        R = cache.get(p)
+        if R is None:
+            R = cache[p] = rope_matrix(*p, D=D, base=base)
+        out[u] = x[u].astype(np.float64) @ R.T
+    return round_to_dtype(out, dtype).astype(np.float32)

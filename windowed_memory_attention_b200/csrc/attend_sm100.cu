@@ -287,8 +287,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // 2^x for two values on the FMA pipe: x = j + f, j = rne(x) through the
 // 1.5*2^23 shifter, p(f) by Horner, then j added to the exponent field.
-// x is clamped to >= -125 so the exponent never underflows into the sign.
+// x is clamped to >= -125 so the exponent never underflows into the sign;
+// an input below -125 (a masked key's -inf among them) gives exactly 0.
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+    const bool z0 = x0 < -125.f, z1 = x1 < -125.f;
     x0 = fmaxf(x0, -125.f);
     x1 = fmaxf(x1, -125.f);
     const uint64_t x = f2(x0, x1);
@@ -303,6 +305,8 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
     unf2(p, p0, p1);
     y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
     y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+    y0 = z0 ? 0.f : y0;
+    y1 = z1 ? 0.f : y1;
 }
 
 // ---------------------------------------------------------------------------
