@@ -37,23 +37,35 @@ def _entries(cache, F):
     return arr, len(lay)
 
 
-def _noalloc(cache, w, layer, q, F, walk, nwalk, **extra):
+KEPT = {gca.GCA_MEMORY_SUMMARY: None, gca.GCA_MEMORY_CAMERA: 1, gca.GCA_MEMORY_NONE: 0}
+
+
+def _noalloc(cache, w, layer, q, F, walk, nwalk, num_pages=None, **extra):
     info = cache.info()
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    kept = KEPT[extra.get("trajectory_memory", gca.GCA_MEMORY_SUMMARY)]
     gca.gca_attend_pages_noalloc(
-        info.k_pool, info.v_pool, num_layers=w.L, num_pages=info.num_pages, num_heads=w.H,
+        info.k_pool, info.v_pool, num_layers=w.L,
+        num_pages=info.num_pages if num_pages is None else num_pages, num_heads=w.H,
         page_size=w.page_size, layer=layer, walk=walk, nwalk=nwalk, q=q, num_query_frames=F,
         tokens_per_frame=w.Lq, first_query_frame=info.frames - F, num_anchor=w.n, window=w.k,
-        summary_tokens=w.S, anchor_block=extra.get("anchor_block", False),
+        summary_tokens=w.S if kept is None else kept, anchor_block=extra.get("anchor_block", False),
         softmax_scale=w.softmax_scale, out=out, lse=lse)
     return out, lse
 
 
-@pytest.mark.parametrize("case", ["tiny", "split_heads", "block3_device_walk"])
+@pytest.mark.parametrize("case", ["tiny", "split_heads", "block3_device_walk", "camera_only",
+                                  "sliding_window"])
 def test_noalloc_matches_gca_attend_on_two_calls(case):
     if case == "tiny":
         w, frames, F, layer, extra = inputs.TINY_BF16, 20, 1, 0, {}
+    elif case == "camera_only":
+        # one kept special token per frame (the camera token)
+        w, frames, F, layer, extra = inputs.TINY_BF16, 20, 1, 0, {"trajectory_memory": gca.GCA_MEMORY_CAMERA}
+    elif case == "sliding_window":
+        # nothing kept and no anchors: the summary-token count is 0
+        w, frames, F, layer, extra = inputs.TINY_BF16.with_(n=0), 20, 1, 0, {"trajectory_memory": gca.GCA_MEMORY_NONE}
     elif case == "split_heads":
         # 546 walk entries x 16 heads over 37 workers: heads are split, so the
         # partials and the merge go through the static scratch
@@ -94,3 +106,36 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
             tokens_per_frame=w.Lq, first_query_frame=0, num_anchor=w.n, window=w.k,
             summary_tokens=w.S, anchor_block=False, softmax_scale=w.softmax_scale, out=q)
     assert e.value.name == "GCA_ERR_CAPACITY"
+
+
+def test_noalloc_rejects_pools_smaller_than_the_sizes_say():
+    # a num_pages past the pools' allocation is refused before any launch
+    w = inputs.TINY_BF16
+    cache = _stream(w, 6)
+    info = cache.info()
+    q = inputs.draw(w, 5, "q", "cuda")
+    walk, nwalk = _entries(cache, 1)
+    with pytest.raises(gca.GCAError) as e:
+        _noalloc(cache, w, 0, q, 1, walk, nwalk, num_pages=info.num_pages * 1000)
+    assert e.value.name == "GCA_ERR_INVALID_ARG"
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+
+
+def test_noalloc_rejects_bad_host_walk_entries():
+    w = inputs.TINY_BF16
+    cache = _stream(w, 6)
+    info = cache.info()
+    q = inputs.draw(w, 5, "q", "cuda")
+    for field, value in (("page_id", info.num_pages), ("page_id", -1), ("n_valid", w.page_size + 1),
+                         ("kind", 7)):
+        walk, nwalk = _entries(cache, 1)
+        setattr(walk[nwalk - 1], field, value)
+        with pytest.raises(gca.GCAError) as e:
+            _noalloc(cache, w, 0, q, 1, walk, nwalk)
+        assert e.value.name == "GCA_ERR_INVALID_ARG", (field, value)
+    # the entries as the cache lists them still work
+    walk, nwalk = _entries(cache, 1)
+    out, _ = _noalloc(cache, w, 0, q, 1, walk, nwalk)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()

@@ -51,7 +51,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
 EncodeTiledFn g_encode = nullptr;
+AddressRangeFn g_range = nullptr;
 
 // Device address of the scratch array on the current device, looked up once
 // per device.
@@ -66,14 +68,17 @@ unsigned char* scratch_address(int dev) {
         }
         g_scratch_addr[dev] = ptr;
     }
-    if (!g_encode) {
+    if (!g_encode || !g_range) {
         void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q{};
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn) {
+        void* fr = nullptr;
+        cudaDriverEntryPointQueryResult q{}, qr{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn ||
+            cudaGetDriverEntryPoint("cuMemGetAddressRange", &fr, cudaEnableDefault, &qr) != cudaSuccess || !fr) {
             cudaGetLastError();
             return nullptr;
         }
         g_encode = (EncodeTiledFn)fn;
+        g_range = (AddressRangeFn)fr;
     }
     return static_cast<unsigned char*>(g_scratch_addr[dev]);
 }
@@ -96,6 +101,17 @@ bool is_device_ptr(const void* ptr) {
     return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
 }
 
+// True when [ptr, ptr + bytes) lies inside the device allocation that holds
+// ptr (for memory from a caching allocator: inside the block it carved ptr
+// from), so that no kernel of this call reads or writes past it.
+bool fits_allocation(const void* ptr, size_t bytes) {
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (!g_range || g_range(&base, &size, (CUdeviceptr)ptr) != CUDA_SUCCESS) return false;
+    const size_t off = (size_t)((CUdeviceptr)ptr - base);
+    return off <= size && bytes <= size - off;
+}
+
 }  // namespace
 
 extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, int32_t num_layers,
@@ -109,7 +125,8 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     if (!k_pool || !v_pool || !walk || !q || !out) return GCA_ERR_INVALID_ARG;
     if (num_layers < 1 || num_pages < 1 || num_heads < 1 || layer < 0 || layer >= num_layers ||
         nwalk < 1 || num_query_frames < 1 || tokens_per_frame < 1 || first_query_frame < 0 ||
-        num_anchor < 0 || window < 1 || summary_tokens < 1 || softmax_scale < 0.f)
+        num_anchor < 0 || window < 1 || summary_tokens < 0 || summary_tokens > tokens_per_frame ||
+        softmax_scale < 0.f)
         return GCA_ERR_INVALID_ARG;
     if (page_size != 64 && page_size != 128) return GCA_ERR_UNSUPPORTED;
     if (!is_device_ptr(k_pool) || !is_device_ptr(v_pool) || !is_device_ptr(q) || !is_device_ptr(out) ||
@@ -127,6 +144,27 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     unsigned char* base = scratch_address(dev);
     if (!base) return GCA_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // every buffer the kernels touch must hold what the sizes say
+    const size_t pool_bytes = (size_t)num_layers * num_pages * num_heads * page_size * gca::kHeadDim * 2;
+    const size_t qo_bytes = (size_t)R * num_heads * gca::kHeadDim * 2;
+    if (!fits_allocation(k_pool, pool_bytes) || !fits_allocation(v_pool, pool_bytes) ||
+        !fits_allocation(q, qo_bytes) || !fits_allocation(out, qo_bytes) ||
+        (lse && !fits_allocation(lse, (size_t)R * num_heads * sizeof(float))) ||
+        (status && !fits_allocation(status, sizeof(int32_t))))
+        return GCA_ERR_INVALID_ARG;
+    const bool walk_on_host = !is_device_ptr(walk);
+    if (walk_on_host) {
+        // a host walk list is checked here; a device one by the kernel (status word)
+        for (int i = 0; i < nwalk; ++i) {
+            const gca_page_entry_t& e = walk[i];
+            if (e.page_id < 0 || e.page_id >= num_pages || e.n_valid < 0 || e.n_valid > page_size ||
+                (e.kind != GCA_PAGE_IMAGE && e.kind != GCA_PAGE_SUMMARY))
+                return GCA_ERR_INVALID_ARG;
+        }
+    } else if (!fits_allocation(walk, sizeof(gca_page_entry_t) * (size_t)nwalk)) {
+        return GCA_ERR_INVALID_ARG;
+    }
     int* d_status = reinterpret_cast<int*>(base);
     gca_page_entry_t* walk_raw = reinterpret_cast<gca_page_entry_t*>(base + kStatusBytes);
     int4* walk_dev = reinterpret_cast<int4*>(base + kStatusBytes + kWalkRawBytes);
@@ -134,7 +172,7 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     float* ws_o = reinterpret_cast<float*>(base + kStatusBytes + kWalkRawBytes + kWalkBytes + kLseBytes);
 
     const gca_page_entry_t* src = walk;
-    if (!is_device_ptr(walk)) {
+    if (walk_on_host) {
         if (cudaMemcpyAsync(walk_raw, walk, sizeof(gca_page_entry_t) * nwalk, cudaMemcpyHostToDevice, st) != cudaSuccess)
             return GCA_ERR_CUDA;
         src = walk_raw;
