@@ -75,6 +75,22 @@ typedef enum { GCA_DTYPE_BF16 = 0, GCA_DTYPE_F32 = 1 } gca_dtype;
  * The special tokens a frame does not keep are stored with its image tokens
  * and leave the cache with them. */
 typedef enum { GCA_MEMORY_SUMMARY = 0, GCA_MEMORY_CAMERA = 1, GCA_MEMORY_NONE = 2 } gca_memory;
+
+/* Position encoding applied inside the library (news article, video RoPE
+ * ablation; paper digest §2.7, a timestamp on the summary tokens; code
+ * walkthrough §3.1, enable_3d_rope):
+ *   NONE  q and k are used as given (already encoded by the caller);
+ *   3D    rotary encoding (RoFormer) over time t, patch row y and patch column
+ *         x: head dims 0..23 rotate with t, 24..43 with y, 44..63 with x; in
+ *         each part of d dims, pair (2i, 2i+1) turns by pos * base^(-2i/d).
+ *         Image token m of frame t sits at (t, m / grid_w, m % grid_w), the
+ *         frame's special tokens at (t, 0, 0); t is the frame's index in the
+ *         cache.  gca_append_frame rotates K as it stores it (the pools hold
+ *         rotated keys, in the cache dtype), the attention calls rotate q as
+ *         they load it; v is not rotated.  A non-keyframe
+ *         (gca_attend_transient) takes the latest keyframe's t; intra-frame
+ *         attention uses t = 0 (only differences of positions matter). */
+typedef enum { GCA_ROPE_NONE = 0, GCA_ROPE_3D = 1 } gca_rope;
 typedef enum { GCA_PAGE_IMAGE = 0, GCA_PAGE_SUMMARY = 1 } gca_page_kind;
 
 typedef struct gca_cache gca_cache_t;  /* opaque, library-owned */
@@ -99,6 +115,9 @@ typedef struct {
     int32_t frame_slack;      /* extra full frames of page space (>= 0)          */
     float softmax_scale;      /* 0 selects 1/sqrt(D)                             */
     int32_t trajectory_memory; /* gca_memory; 0 (SUMMARY) is GCA                 */
+    int32_t rope;             /* gca_rope: 3D rotary position encoding of Q, K   */
+    int32_t rope_grid_w;      /* patch columns of the image-token grid (0: M)    */
+    float rope_base;          /* rotary base (0 selects 10000)                   */
 } gca_config_t;
 
 /* One entry of the walk list (the pages gca_attend reads, in order).  Below,
@@ -274,11 +293,22 @@ const char* gca_status_string(int status);
  * float32 (device, nullable) and status (device int, nullable: raised like
  * the cache's status word).  summary_tokens is the number of special tokens
  * each frame keeps in the summary stream (s_k: S, 1 or 0 by the cache's
- * trajectory_memory).  Scratch lives in one static device array of
- * 18 MiB per GPU: at most 32768 walk entries and 512 partial tiles of 128
- * query rows (ceil(F*Lq/128) * H <= 512), else GCA_ERR_CAPACITY.  The first
- * call on a device looks up the array's address (call it before any stream
- * capture); calls whose GPU work overlaps share the array and race. */
+ * trajectory_memory; 0 <= s_k <= tokens_per_frame).
+ * Checks before any launch (INVALID_ARG): every device buffer must lie inside
+ * its allocation for the sizes given (the pools for num_layers * num_pages
+ * pages, q and out for F * tokens_per_frame rows, lse, status, a device walk
+ * list); a host walk list must hold page ids in [0, num_pages), n_valid in
+ * [0, page_size] and a known kind.  A device walk list is checked by the
+ * kernel, which raises *status on a bad page id.  With status = NULL a
+ * device-side failure (a bad page id in a device walk list, a bounded wait
+ * that ran out) is not reported to the caller, and out may be left unwritten.
+ * A real-time caller should pass the walk list in device or pinned host
+ * memory: a pageable host list is staged by a copy that can block the host.
+ * Scratch lives in one static device array of 18 MiB per GPU: at most 32768
+ * walk entries and 512 partial tiles of 128 query rows
+ * (ceil(F*Lq/128) * H <= 512), else GCA_ERR_CAPACITY.  The first call on a
+ * device looks up the array's address (call it before any stream capture);
+ * calls whose GPU work overlaps share the array and race. */
 int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, int32_t num_layers,
                              int32_t num_pages, int32_t num_heads, int32_t page_size,
                              int32_t layer, const gca_page_entry_t* walk, int32_t nwalk,

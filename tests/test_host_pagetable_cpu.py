@@ -197,3 +197,28 @@ def test_null_and_range_arguments_are_rejected():
     assert err.value.name == "GCA_ERR_INVALID_ARG"
     assert L.gca_cache_destroy(None) == 0            # null is accepted
     cache.close()
+
+
+def test_walk_list_is_the_same_before_and_after_the_eviction():
+    # gca_attend may run with the step's eviction still pending: for a single
+    # query frame the walk list holds only the frames it may see, so it does
+    # not change when the frame that left the window gives back its pages
+    w = inputs.METRIC_518x378.with_(L=1)
+    cache, sim = _pair(w)
+    for t in range(200):
+        assert cache.append(None, None) == sim.append()
+        before = cache.layout()
+        n = cache.evict()
+        assert n == sim.evict() == (1 if t >= w.n + w.k else 0)
+        assert cache.layout() == before == sim.walk()
+
+
+def test_rope_configuration_is_checked():
+    w = inputs.TINY
+    for bad in ({"rope": 2}, {"rope": -1}, {"rope": gca.GCA_ROPE_3D, "rope_grid_w": -1},
+                {"rope": gca.GCA_ROPE_3D, "rope_base": -5.0}):
+        with pytest.raises(gca.GCAError) as e:
+            gca.Cache.for_workload(w, device=gca.GCA_HOST_ONLY, **bad)
+        assert e.value.name == "GCA_ERR_INVALID_ARG"
+    c = gca.Cache.for_workload(w, device=gca.GCA_HOST_ONLY, rope=gca.GCA_ROPE_3D, rope_grid_w=4)
+    assert c.append(None, None) == 0

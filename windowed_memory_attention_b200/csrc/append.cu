@@ -15,6 +15,13 @@
 // Slots that no token fills (the tail of a frame's last image page, and the
 // not-yet-used tail of a newly opened summary page) are zeroed, so a masked
 // key never multiplies stale non-finite bytes in the PV product.
+//
+// With the 3D rotary encoding on, K is rotated as it is stored: each dim pair
+// (2i, 2i+1) of token u turns by the angle of its axis (frame time for pairs
+// 0..11, patch row and column for 12..31), in fp32, and is rounded back to
+// the cache dtype (see RopeTables).
+#include <cuda_bf16.h>
+
 #include "gca_internal.h"
 
 namespace gca {
@@ -68,13 +75,15 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     const unsigned n_zsum = H * sum_tail * cpr;
     const unsigned total = n_copy + n_zimg + n_zsum;
 
-    // destination of chunk u (and whether it is a zero fill)
-    auto dest = [&](unsigned u, bool& zero) -> char* {
+    // destination of chunk u (and whether it is a zero fill); tok / chunk: the
+    // chunk's token in the frame and its 16-byte index within the head's row
+    auto dest = [&](unsigned u, bool& zero, unsigned& tok, unsigned& chunk) -> char* {
         if (u < n_copy) {
             zero = false;
-            const unsigned chunk = u & (cpr - 1);
+            chunk = u & (cpr - 1);
             const unsigned th = u >> cpr_shift;
             const unsigned tau = HSHIFT >= 0 ? th >> HSHIFT : th / H;
+            tok = tau;
             const unsigned h = HSHIFT >= 0 ? th & ((1u << (HSHIFT & 31)) - 1u) : th - tau * H;
             int page, slot;
             if ((int)tau < p.S) {
@@ -91,6 +100,8 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
                    (long long)slot * row_bytes + chunk * 16;
         }
         zero = true;
+        tok = 0;
+        chunk = 0;
         unsigned z = u - n_copy;
         int page;
         unsigned slot0, nslots;
@@ -104,12 +115,33 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
             slot0 = sum_from;
             nslots = sum_tail;
         }
-        const unsigned chunk = z & (cpr - 1);
+        const unsigned zc = z & (cpr - 1);
         const unsigned ts = z >> cpr_shift;
         const unsigned h = ts / nslots;
         const unsigned sl = ts - h * nslots;
         return lpool + ((long long)page * p.H + h) * tile_bytes +
-               (long long)(slot0 + sl) * row_bytes + chunk * 16;
+               (long long)(slot0 + sl) * row_bytes + zc * 16;
+    };
+    // K with the 3D rotary encoding: each 16-byte chunk holds whole dim pairs
+    const bool rotate = tensor == 0 && p.rope.t != nullptr;
+    auto rope_chunk = [&](int4& v, unsigned tok, unsigned chunk) {
+        if (p.elem_bytes == 2) {
+            uint32_t w[4] = {(uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 b2 = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
+                float a = __low2float(b2), b = __high2float(b2);
+                rope_rotate(a, b, rope_cs(p.rope, p.rope_t, (int)tok, (int)chunk * 4 + j));
+                b2 = __floats2bfloat162_rn(a, b);
+                w[j] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            v = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
+        } else {
+            float f[4] = {__int_as_float(v.x), __int_as_float(v.y), __int_as_float(v.z), __int_as_float(v.w)};
+            rope_rotate(f[0], f[1], rope_cs(p.rope, p.rope_t, (int)tok, (int)chunk * 2));
+            rope_rotate(f[2], f[3], rope_cs(p.rope, p.rope_t, (int)tok, (int)chunk * 2 + 1));
+            v = make_int4(__float_as_int(f[0]), __float_as_int(f[1]), __float_as_int(f[2]), __float_as_int(f[3]));
+        }
     };
 
     // four independent chunks per thread per iteration: loads first, then stores
@@ -119,15 +151,21 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         int4 val[U];
         char* dst[U];
         bool zero[U];
+        unsigned tok[U], chunk[U];
 #pragma unroll
         for (int i = 0; i < U; ++i) {
             const unsigned u = base + i * stride;
             dst[i] = nullptr;
             if (u < total) {
-                dst[i] = dest(u, zero[i]);
+                dst[i] = dest(u, zero[i], tok[i], chunk[i]);
                 val[i] = zero[i] ? make_int4(0, 0, 0, 0)
                                  : ld_stream(reinterpret_cast<const int4*>(src) + u);
             }
+        }
+        if (rotate) {
+#pragma unroll
+            for (int i = 0; i < U; ++i)
+                if (dst[i] && !zero[i]) rope_chunk(val[i], tok[i], chunk[i]);
         }
 #pragma unroll
         for (int i = 0; i < U; ++i)

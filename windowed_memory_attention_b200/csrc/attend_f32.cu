@@ -29,9 +29,16 @@ attend_f32_kernel(const AttendParams p, const float* __restrict__ kpool,
     const float* qg = static_cast<const float*>(p.q) + ((long long)(valid ? row : 0) * p.H + h) * kHeadDim;
 #pragma unroll
     for (int d = 0; d < kHeadDim; ++d) {
-        q[d] = valid ? qg[d] * p.scale : 0.f;
+        q[d] = valid ? qg[d] : 0.f;
         acc[d] = 0.f;
     }
+    if (p.rope.t) {      // 3D rotary encoding of the query at its frame's position
+        const int u = valid ? row % p.Lq : 0;
+#pragma unroll
+        for (int i = 0; i < kHeadDim / 2; ++i) rope_rotate(q[2 * i], q[2 * i + 1], rope_cs(p.rope, qframe, u, i));
+    }
+#pragma unroll
+    for (int d = 0; d < kHeadDim; ++d) q[d] *= p.scale;
     float m = -INFINITY, l = 0.f;
     const long long tile = (long long)p.P * kHeadDim;
     for (int e = 0; e < p.nwalk; ++e) {

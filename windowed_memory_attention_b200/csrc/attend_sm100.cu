@@ -519,6 +519,18 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     r[4 * i + 2] = v.z;
                     r[4 * i + 3] = v.w;
                 }
+                if (p.rope.t) {
+                    // 3D rotary encoding at the row's (frame, token) position:
+                    // each 32-bit word holds dim pair i in fp32, rounded back to bf16
+                    const int u = row % p.Lq;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        __nv_bfloat162 b2 = *reinterpret_cast<__nv_bfloat162*>(&r[i]);
+                        float a = __low2float(b2), b = __high2float(b2);
+                        rope_rotate(a, b, rope_cs(p.rope, qframe, u, i));
+                        r[i] = pack_bf16(a, b);
+                    }
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) r[i] = 0u;

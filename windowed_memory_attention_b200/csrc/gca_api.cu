@@ -41,6 +41,7 @@ using gca::WalkEntry;
 namespace {
 
 constexpr int kRing = 4;       // pinned staging slots for walk-list uploads
+constexpr int kQRing = 4;      // device staging slots for host query blocks
 constexpr int kTileRows = 128;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -95,14 +96,26 @@ struct gca_cache {
     size_t ws_slots = 0;
     int* h_status = nullptr;
     int* d_status = nullptr;
-    // staging for host-memory arguments
+    // staging for host-memory arguments: inputs are copied on the library's own
+    // copy stream (so uploads overlap the caller's compute stream), guarded by
+    // events; pinned host outputs are written by the kernels directly
+    cudaStream_t copy = nullptr;
     void* st_k = nullptr;
     void* st_v = nullptr;
-    void* st_q = nullptr;
+    cudaEvent_t kv_free = nullptr, kv_ready = nullptr;
+    void* st_q[kQRing] = {};
+    cudaEvent_t q_free[kQRing] = {}, q_ready[kQRing] = {};
+    int q_pos = 0;
     void* st_out = nullptr;
     float* st_lse = nullptr;
     long long launches = 0;
     bool host_only = false;   // GCA_HOST_ONLY: the page table alone, no device state
+    // 3D rotary encoding: (cos, sin) tables of the time pairs per frame index
+    // and of the spatial pairs per token of a frame
+    float2* rope_t = nullptr;
+    float2* rope_sp = nullptr;
+    int rope_max_t = 0;
+    gca::RopeTables rope() const { return {rope_t, rope_sp, rope_max_t}; }
 };
 
 namespace {
@@ -126,9 +139,18 @@ void release(gca_cache* c) {
     cudaFree(c->ws_lse);
     cudaFree(c->st_k);
     cudaFree(c->st_v);
-    cudaFree(c->st_q);
+    for (int i = 0; i < kQRing; ++i) {
+        cudaFree(c->st_q[i]);
+        if (c->q_free[i]) cudaEventDestroy(c->q_free[i]);
+        if (c->q_ready[i]) cudaEventDestroy(c->q_ready[i]);
+    }
     cudaFree(c->st_out);
     cudaFree(c->st_lse);
+    cudaFree(c->rope_t);
+    cudaFree(c->rope_sp);
+    if (c->kv_free) cudaEventDestroy(c->kv_free);
+    if (c->kv_ready) cudaEventDestroy(c->kv_ready);
+    if (c->copy) cudaStreamDestroy(c->copy);
     for (int i = 0; i < kRing; ++i) {
         if (c->h_stage[i]) cudaFreeHost(c->h_stage[i]);
         if (c->stage_ev[i]) cudaEventDestroy(c->stage_ev[i]);
@@ -161,13 +183,56 @@ struct DeviceGuard {
     }
 };
 
-bool is_device_ptr(const void* ptr) {
+// Where a caller's pointer lives: device memory (used as is), pinned host
+// memory (the device reaches it through *alias), or pageable host memory.
+enum class Mem { kDevice, kPinned, kPageable };
+
+Mem classify(const void* ptr, void** alias = nullptr) {
     cudaPointerAttributes a{};
     if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
         cudaGetLastError();
-        return false;
+        return Mem::kPageable;
     }
-    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return Mem::kDevice;
+    if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+        if (alias) *alias = a.devicePointer;
+        return Mem::kPinned;
+    }
+    return Mem::kPageable;
+}
+
+bool is_device_ptr(const void* ptr) { return classify(ptr) == Mem::kDevice; }
+
+// Upload a host input into a staging buffer on the cache's copy stream: the
+// copy waits until the buffer's previous reader (on the caller's stream) is
+// done (`free_ev`), and the caller's stream waits for the copy (`ready_ev`).
+// The caller records free_ev on its stream after the kernel that reads dst.
+bool stage_in(gca_cache* c, void* dst, const void* src, size_t bytes, cudaEvent_t free_ev,
+              cudaEvent_t ready_ev, cudaStream_t st) {
+    return cudaStreamWaitEvent(c->copy, free_ev, 0) == cudaSuccess &&
+           cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, c->copy) == cudaSuccess &&
+           cudaEventRecord(ready_ev, c->copy) == cudaSuccess &&
+           cudaStreamWaitEvent(st, ready_ev, 0) == cudaSuccess;
+}
+
+// K and V of a frame (or of all layers) from the caller, staged when on the host.
+bool stage_kv(gca_cache* c, const void* k, const void* v, size_t bytes, cudaStream_t st,
+              const void** kd, const void** vd) {
+    *kd = k;
+    *vd = v;
+    const bool kh = !is_device_ptr(k), vh = !is_device_ptr(v);
+    if (!kh && !vh) return true;
+    if (cudaStreamWaitEvent(c->copy, c->kv_free, 0) != cudaSuccess) return false;
+    if (kh) {
+        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, c->copy) != cudaSuccess) return false;
+        *kd = c->st_k;
+    }
+    if (vh) {
+        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, c->copy) != cudaSuccess) return false;
+        *vd = c->st_v;
+    }
+    return cudaEventRecord(c->kv_ready, c->copy) == cudaSuccess &&
+           cudaStreamWaitEvent(st, c->kv_ready, 0) == cudaSuccess;
 }
 
 bool encode_pool_map(EncodeTiledFn enc, CUtensorMap* tm, void* pool, const gca_cache* c) {
@@ -180,6 +245,38 @@ bool encode_pool_map(EncodeTiledFn enc, CUtensorMap* tm, void* pool, const gca_c
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
+}
+
+// Host tables of the 3D rotary encoding.  Axis a (time, patch row, patch
+// column) owns d_a = 24, 20, 20 head dims; its pair i turns by
+// pos * base^(-2i/d_a).  Angles are formed in double and stored as float.
+bool build_rope_tables(gca_cache* c) {
+    const gca_config_t& g = c->cfg;
+    const double base = g.rope_base > 0.f ? (double)g.rope_base : 10000.0;
+    const int gw = g.rope_grid_w > 0 ? g.rope_grid_w : g.image_tokens;
+    auto freq = [&](int i, int d) { return std::pow(base, -2.0 * i / d); };
+    c->rope_max_t = g.max_frames;
+    std::vector<float2> ht((size_t)c->rope_max_t * gca::kRopeTPairs);
+    for (int t = 0; t < c->rope_max_t; ++t)
+        for (int i = 0; i < gca::kRopeTPairs; ++i) {
+            const double a = t * freq(i, 2 * gca::kRopeTPairs);
+            ht[(size_t)t * gca::kRopeTPairs + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+        }
+    std::vector<float2> hs((size_t)c->Lq * gca::kRopeSpPairs);
+    constexpr int kYPairs = gca::kRopeSpPairs / 2;         // 10 pairs each for row and column
+    for (int u = 0; u < c->Lq; ++u) {
+        const int m = u - g.summary_tokens;                 // image token index, < 0: special
+        const int y = m < 0 ? 0 : m / gw, x = m < 0 ? 0 : m % gw;
+        for (int i = 0; i < gca::kRopeSpPairs; ++i) {
+            const int pos = i < kYPairs ? y : x;
+            const double a = pos * freq(i % kYPairs, 2 * kYPairs);
+            hs[(size_t)u * gca::kRopeSpPairs + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+        }
+    }
+    return cudaMalloc(&c->rope_t, ht.size() * sizeof(float2)) == cudaSuccess &&
+           cudaMalloc(&c->rope_sp, hs.size() * sizeof(float2)) == cudaSuccess &&
+           cudaMemcpy(c->rope_t, ht.data(), ht.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
+           cudaMemcpy(c->rope_sp, hs.data(), hs.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess;
 }
 
 bool frame_seen(const gca_cache* c, int i, int j) {
@@ -239,19 +336,31 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     const int R = F * c->Lq;
     const size_t qbytes = (size_t)R * g.num_heads * gca::kHeadDim * c->elem;
     const void* qd = q;
+    int qslot = -1;
     if (!is_device_ptr(q)) {
-        if (cudaMemcpyAsync(c->st_q, q, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        qd = c->st_q;
+        qslot = c->q_pos;
+        c->q_pos = (c->q_pos + 1) % kQRing;
+        if (!stage_in(c, c->st_q[qslot], q, qbytes, c->q_free[qslot], c->q_ready[qslot], st))
+            return GCA_ERR_CUDA;
+        qd = c->st_q[qslot];
     }
-    const bool out_host = !is_device_ptr(out);
-    const bool lse_host = lse && !is_device_ptr(lse);
+    // outputs: device memory and pinned host memory (through its device alias)
+    // are written by the kernels; pageable host memory is staged and copied back
+    void* out_alias = nullptr;
+    void* lse_alias = nullptr;
+    const Mem out_mem = classify(out, &out_alias);
+    const Mem lse_mem = lse ? classify(lse, &lse_alias) : Mem::kDevice;
+    const bool out_host = out_mem == Mem::kPageable;
+    const bool lse_host = lse && lse_mem == Mem::kPageable;
+    void* out_k = out_mem == Mem::kPinned ? out_alias : out;
+    float* lse_k = lse_mem == Mem::kPinned ? static_cast<float*>(lse_alias) : lse;
 
     gca::AttendParams p{};
     p.walk = walk;
     p.nwalk = nwalk;
     p.q = qd;
-    p.out = out_host ? c->st_out : out;
-    p.lse = lse ? (lse_host ? c->st_lse : lse) : nullptr;
+    p.out = out_host ? c->st_out : out_k;
+    p.lse = lse ? (lse_host ? c->st_lse : lse_k) : nullptr;
     p.R = R;
     p.H = g.num_heads;
     p.Lq = c->Lq;
@@ -265,6 +374,7 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     p.status = c->d_status;
     p.ws_o = c->ws_o;
     p.ws_lse = c->ws_lse;
+    p.rope = c->rope();
 
     cudaError_t err;
     if (g.dtype == GCA_DTYPE_BF16) {
@@ -296,6 +406,7 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
         cudaGetLastError();
         return GCA_ERR_CUDA;
     }
+    if (qslot >= 0 && cudaEventRecord(c->q_free[qslot], st) != cudaSuccess) return GCA_ERR_CUDA;
     if (out_host && cudaMemcpyAsync(out, c->st_out, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return GCA_ERR_CUDA;
     if (lse_host && cudaMemcpyAsync(lse, c->st_lse, (size_t)R * g.num_heads * sizeof(float),
@@ -310,16 +421,7 @@ int stage_transient(gca_cache* c, int layer, const void* k, const void* v, int f
     const gca_config_t& g = c->cfg;
     gca::AppendParams p{};
     const size_t bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
-    p.k = k;
-    p.v = v;
-    if (!is_device_ptr(k)) {
-        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        p.k = c->st_k;
-    }
-    if (!is_device_ptr(v)) {
-        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        p.v = c->st_v;
-    }
+    if (!stage_kv(c, k, v, bytes, st, &p.k, &p.v)) return GCA_ERR_CUDA;
     p.kpool = c->kpool;
     p.vpool = c->vpool;
     p.layer0 = layer;
@@ -337,11 +439,14 @@ int stage_transient(gca_cache* c, int layer, const void* k, const void* v, int f
     p.sum_page[0] = p.sum_page[1] = -1;
     p.new_sum_seq = -1;
     for (int s = 0; s < c->tpf; ++s) p.img_pages[s] = c->num_regular + s;
+    p.rope = c->rope();
+    p.rope_t = frame;
     if (gca::launch_append(p, st) != cudaSuccess) {
         cudaGetLastError();
         return GCA_ERR_CUDA;
     }
     c->launches += 1;
+    if (cudaEventRecord(c->kv_free, st) != cudaSuccess) return GCA_ERR_CUDA;
     return GCA_OK;
 }
 
@@ -373,7 +478,8 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     if (g.num_layers < 1 || g.num_heads < 1 || g.image_tokens < 1 || g.summary_tokens < 1 ||
         g.num_anchor < 0 || g.window < 1 || g.max_frames < 1 || g.max_query_frames < 1 ||
         g.frame_slack < 0 || g.softmax_scale < 0.f || g.trajectory_memory < GCA_MEMORY_SUMMARY ||
-        g.trajectory_memory > GCA_MEMORY_NONE)
+        g.trajectory_memory > GCA_MEMORY_NONE || g.rope < GCA_ROPE_NONE || g.rope > GCA_ROPE_3D ||
+        g.rope_grid_w < 0 || g.rope_base < 0.f)
         return GCA_ERR_INVALID_ARG;
     if (g.head_dim != gca::kHeadDim || (g.page_size != 64 && g.page_size != 128) ||
         (g.dtype != GCA_DTYPE_BF16 && g.dtype != GCA_DTYPE_F32))
@@ -451,12 +557,23 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
         ok = cudaHostGetDevicePointer((void**)&c->d_status, c->h_status, 0) == cudaSuccess;
     }
     const size_t frame_bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
+    ok = ok && cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->kv_free, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->kv_ready, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < kQRing; ++i)
+        ok = cudaMalloc(&c->st_q[i], frame_bytes * g.max_query_frames) == cudaSuccess &&
+             cudaEventCreateWithFlags(&c->q_free[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&c->q_ready[i], cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaMalloc(&c->st_k, frame_bytes * g.num_layers) == cudaSuccess &&
          cudaMalloc(&c->st_v, frame_bytes * g.num_layers) == cudaSuccess &&
-         cudaMalloc(&c->st_q, frame_bytes * g.max_query_frames) == cudaSuccess &&
          cudaMalloc(&c->st_out, frame_bytes * g.max_query_frames) == cudaSuccess &&
          cudaMalloc((void**)&c->st_lse, (size_t)c->Lq * g.num_heads * g.max_query_frames * sizeof(float)) == cudaSuccess;
     if (!ok) {
+        cudaGetLastError();
+        release(c);
+        return GCA_ERR_CUDA;
+    }
+    if (g.rope == GCA_ROPE_3D && !build_rope_tables(c)) {
         cudaGetLastError();
         release(c);
         return GCA_ERR_CUDA;
@@ -532,16 +649,7 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
 
     gca::AppendParams p{};
     const size_t bytes = (size_t)nl * c->Lq * g.num_heads * gca::kHeadDim * c->elem;
-    p.k = k;
-    p.v = v;
-    if (!is_device_ptr(k)) {
-        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        p.k = c->st_k;
-    }
-    if (!is_device_ptr(v)) {
-        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GCA_ERR_CUDA;
-        p.v = c->st_v;
-    }
+    if (!stage_kv(c, k, v, bytes, st, &p.k, &p.v)) return GCA_ERR_CUDA;
     p.kpool = c->kpool;
     p.vpool = c->vpool;
     p.layer0 = l0;
@@ -564,11 +672,14 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
         if (((S * t + s) % c->P) == 0) p.new_sum_seq = (S * t + s) / c->P;
     const std::vector<int>& img = c->image_pages.at(t);
     for (int i = 0; i < c->ipf; ++i) p.img_pages[i] = img[i];
+    p.rope = c->rope();
+    p.rope_t = t;
     if (gca::launch_append(p, st) != cudaSuccess) {
         cudaGetLastError();
         return GCA_ERR_CUDA;
     }
     c->launches += 1;
+    if (cudaEventRecord(c->kv_free, st) != cudaSuccess) return GCA_ERR_CUDA;
     for (int l = l0; l < l0 + nl; ++l) c->layer_frames[l] = t + 1;
     if (frame_index_out) *frame_index_out = t;
     return GCA_OK;

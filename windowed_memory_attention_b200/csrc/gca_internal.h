@@ -40,6 +40,33 @@ __host__ __device__ inline int visible_prefix(const MaskRule& r, int4 e, int i) 
     return v < e.y ? v : e.y;
 }
 
+// 3D rotary encoding tables (cos, sin) of the 32 dim pairs of a head: pairs
+// 0..11 turn with the frame's time index (rope_t[t * 12 + i]), pairs 12..31
+// with the token's patch row and column (rope_sp[u * 20 + i - 12], u = the
+// token's index in its frame, special tokens first).
+constexpr int kRopeTPairs = 12;
+constexpr int kRopeSpPairs = 20;
+
+struct RopeTables {
+    const float2* t;          // [max_t][12], or null: no rotation
+    const float2* sp;         // [S+M][20]
+    int max_t;                // rows of t
+};
+
+#ifdef __CUDACC__
+// (cos, sin) of dim pair i (0..31) for token u of a frame at time index t
+__device__ __forceinline__ float2 rope_cs(const RopeTables& r, int t, int u, int i) {
+    t = t < r.max_t ? t : r.max_t - 1;
+    return i < kRopeTPairs ? r.t[t * kRopeTPairs + i] : r.sp[u * kRopeSpPairs + (i - kRopeTPairs)];
+}
+// (a, b) -> (a cos - b sin, a sin + b cos)
+__device__ __forceinline__ void rope_rotate(float& a, float& b, float2 cs) {
+    const float a2 = fmaf(a, cs.x, -b * cs.y);
+    b = fmaf(a, cs.y, b * cs.x);
+    a = a2;
+}
+#endif
+
 struct AppendParams {
     const void* k;            // [nlayers][Lq][H][D]
     const void* v;
@@ -53,6 +80,8 @@ struct AppendParams {
     int new_sum_seq;          // summary sequence opened by this frame, -1 if none
     int img_pages[kMaxImagePages];
     int sms;                  // SMs of the device (grid sizing)
+    RopeTables rope;          // K of tensor 0 is rotated when rope.t is set
+    int rope_t;               // time index of the frame
 };
 
 struct AttendParams {
@@ -72,6 +101,7 @@ struct AttendParams {
     float* ws_o;              // [QT*(W+H-1)][128][D] partial outputs (normalised)
     float* ws_lse;            // [QT*(W+H-1)][128] partial log2-sum-exp
     int* status;              // device status word (host-mapped)
+    RopeTables rope;          // q rotated on load when rope.t is set
 };
 
 // launchers (return cudaError_t of the launch)

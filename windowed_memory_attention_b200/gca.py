@@ -22,6 +22,7 @@ GCA_HOST_ONLY = -1        # cache-create device: the page table alone (no GPU ne
 GCA_DTYPE_BF16, GCA_DTYPE_F32 = 0, 1
 GCA_PAGE_IMAGE, GCA_PAGE_SUMMARY = 0, 1
 GCA_MEMORY_SUMMARY, GCA_MEMORY_CAMERA, GCA_MEMORY_NONE = 0, 1, 2
+GCA_ROPE_NONE, GCA_ROPE_3D = 0, 1
 STATUS = {0: "GCA_OK", 1: "GCA_ERR_INVALID_ARG", 2: "GCA_ERR_CAPACITY", 3: "GCA_ERR_STATE",
           4: "GCA_ERR_UNSUPPORTED", 5: "GCA_ERR_CUDA", 6: "GCA_ERR_DEVICE_CHECK"}
 EXPORTS = ("gca_cache_create", "gca_cache_destroy", "gca_append_frame", "gca_evict_to_summary",
@@ -35,7 +36,9 @@ class gca_config_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_layers", "num_heads", "head_dim", "image_tokens", "summary_tokens", "num_anchor",
         "window", "max_frames", "page_size", "dtype", "anchor_block", "max_query_frames",
-        "frame_slack")] + [("softmax_scale", ctypes.c_float), ("trajectory_memory", ctypes.c_int32)]
+        "frame_slack")] + [("softmax_scale", ctypes.c_float), ("trajectory_memory", ctypes.c_int32),
+                           ("rope", ctypes.c_int32), ("rope_grid_w", ctypes.c_int32),
+                           ("rope_base", ctypes.c_float)]
 
 
 class gca_page_entry_t(ctypes.Structure):
@@ -127,12 +130,13 @@ def gca_cache_create(*, num_layers: int, num_heads: int, image_tokens: int, num_
                      page_size: int = 128, dtype: str = "bf16", anchor_block: bool = False,
                      max_query_frames: int = 1, frame_slack: int = 0,
                      softmax_scale: float = 0.0, trajectory_memory: int = GCA_MEMORY_SUMMARY,
+                     rope: int = GCA_ROPE_NONE, rope_grid_w: int = 0, rope_base: float = 0.0,
                      device: int = 0) -> ctypes.c_void_p:
     cfg = gca_config_t(num_layers, num_heads, head_dim, image_tokens, summary_tokens, num_anchor,
                        window, max_frames, page_size,
                        GCA_DTYPE_BF16 if dtype == "bf16" else GCA_DTYPE_F32,
                        int(bool(anchor_block)), max_query_frames, frame_slack, softmax_scale,
-                       trajectory_memory)
+                       trajectory_memory, rope, rope_grid_w, rope_base)
     h = ctypes.c_void_p()
     _check("gca_cache_create", lib().gca_cache_create(ctypes.byref(cfg), device, ctypes.byref(h)))
     return h
