@@ -409,7 +409,8 @@ def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, r
             transient=False):
     """Stream frames frame0..frame0+T-1 (local indices 0..T-1); at each local
     step in `checks` compare sampled rows of the listed layers with the oracle
-    (and, with `transient`, a non-keyframe's attention at that state)."""
+    (and, with `transient`, a non-keyframe's attention at that state).  `rows`
+    is a list of token rows, None for every row, or a dict layer -> either."""
     dev = "cuda"
     if reset:
         cache.reset()
@@ -429,10 +430,12 @@ def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, r
             assert cache.layout() == sim.walk()
             q = inputs.draw(w, g, "q", dev)
             for l in layers_to_check:
+                lrows = rows.get(l) if isinstance(rows, dict) else rows
+                sel = slice(None) if lrows is None else lrows
                 out, lse = attend(cache, l, q[l:l + 1].contiguous())
                 torch.cuda.synchronize()
-                want, wlse = oracle_step(mirror, l, q[l:l + 1].float().cpu().numpy(), t, rows=rows)
-                got, gl = out[0][rows], lse[0][rows]
+                want, wlse = oracle_step(mirror, l, q[l:l + 1].float().cpu().numpy(), t, rows=lrows)
+                got, gl = out[0][sel], lse[0][sel]
                 if heads is not None:
                     got, gl = got[:, heads], gl[:, heads]
                 e = max_err(got, want[0])
@@ -447,8 +450,8 @@ def _stream(w, cache, sim, mirror, T, checks, layers_to_check, rows, frame0=0, r
                     out, lse = attend_transient(cache, l, qt, kt, vt)
                     torch.cuda.synchronize()
                     want, wlse = oracle_transient(mirror, l, qt.float().cpu().numpy(), kt.float().cpu().numpy(),
-                                                  vt.float().cpu().numpy(), t, rows=rows)
-                    got, gl = out[rows], lse[rows]
+                                                  vt.float().cpu().numpy(), t, rows=lrows)
+                    got, gl = out[sel], lse[sel]
                     if heads is not None:
                         got, gl = got[:, heads], gl[:, heads]
                     e = max_err(got, want)
@@ -474,11 +477,12 @@ def test_worked_example_to_T10000():
 
 
 def test_metric_workload_T10000_all_layers():
+    # layer 0 in full (all 1005 rows x 16 heads) at T=10000, layer 23 on sampled rows
     w = inputs.METRIC_518x378
     cache = gca.Cache.for_workload(w)
     sim = _sim(w)
     mirror = Mirror(w, [0, 23])
-    rows = _rows_sample(w.Lq, extra=8, seed=3)
+    rows = {0: None, 23: _rows_sample(w.Lq, extra=8, seed=3)}
     res = _stream(w, cache, sim, mirror, w.T, {9999}, [0, 23], rows, transient=True)
     assert cache.info().resident_tokens == 999 * 67 + 6 * 10000
     # every layer's output at T=10000 is finite and its lse lies within the
@@ -491,18 +495,26 @@ def test_metric_workload_T10000_all_layers():
     print("metric workload max errors", res)
 
 
-def test_windowed_vo_windows():
+def test_windowed_vo_full_stream():
+    """The windowed (VO) workload as defined: 179 windows of 128 frames
+    overlapping by 16 over 20,000 frames (22,848 frames processed), a reset at
+    each window start, the window's first n frames its anchors.  Page tables
+    match the simulator at every checked step of every window; sampled rows of
+    two heads match the oracle at steps 0, 2, 66 and the window's last step."""
     w = inputs.WINDOWED_VO
     wins = w.windows()
+    assert len(wins) == 179 and sum(ln for _, ln in wins) == 22848
     cache = gca.Cache.for_workload(w)
     sim = _sim(w)
-    rows = _rows_sample(w.Lq, extra=4, seed=5)
-    checks = {0, 1, 2, 3, 66, 67, 68, 127}
-    for idx in (0, 1, len(wins) - 1):
-        start, ln = wins[idx]
-        mirror = Mirror(w, [0])
-        _stream(w, cache, sim, mirror, ln, {c for c in checks if c < ln}, [0], rows,
-                frame0=start, reset=True)
+    rows = _rows_sample(w.Lq, extra=2, seed=5)
+    processed = 0
+    for idx, (start, ln) in enumerate(wins):
+        mirror = Mirror(w, [0], heads=[idx % w.H, (idx * 7 + 3) % w.H])
+        checks = {c for c in (0, 2, 66, ln - 1) if c < ln}
+        _stream(w, cache, sim, mirror, ln, checks, [0], rows, frame0=start, reset=True)
+        processed += ln
+        assert cache.info().frames == ln
+    assert processed == 22848
 
 
 def test_dense_causal_limit_T1000():
