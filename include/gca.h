@@ -304,7 +304,8 @@ const char* gca_status_string(int status);
  * that ran out) is not reported to the caller, and out may be left unwritten.
  * A real-time caller should pass the walk list in device or pinned host
  * memory: a pageable host list is staged by a copy that can block the host.
- * Scratch lives in one static device array of 18 MiB per GPU: at most 32768
+ * Scratch (split-head partials and their counters, a device copy of the walk
+ * list) lives in one static device array of 18 MiB per GPU: at most 32768
  * walk entries and 512 partial tiles of 128 query rows
  * (ceil(F*Lq/128) * H <= 512), else GCA_ERR_CAPACITY.  The first call on a
  * device looks up the array's address (call it before any stream capture);

@@ -13,8 +13,8 @@
   weight 2^80 too large.
 * Masked key slots: slots past a page's stored tokens carry stale bytes.  The
   tests fill them with the largest finite bf16 value in K and V; a masked key
-  must get weight exactly 0 on every exponential path (MUFU and polynomial
-  lanes alike), so the output still matches the oracle.
+  must get weight exactly 0 (its score is -inf before the exponential), so the
+  output still matches the oracle.
 * Attending before or after gca_evict_to_summary gives identical bytes: the
   walk list holds only the frames the query block may see.
 """

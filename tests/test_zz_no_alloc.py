@@ -68,7 +68,7 @@ def test_noalloc_matches_gca_attend_on_two_calls(case):
         w, frames, F, layer, extra = inputs.TINY_BF16.with_(n=0), 20, 1, 0, {"trajectory_memory": gca.GCA_MEMORY_NONE}
     elif case == "split_heads":
         # 546 walk entries x 16 heads over 37 workers: heads are split, so the
-        # partials and the merge go through the static scratch
+        # partials and their counters go through the static scratch
         w, frames, F, layer, extra = inputs.METRIC_518x378.with_(L=2, T=200), 200, 1, 1, {}
     else:
         w, frames, F, layer, extra = inputs.TINY_BF16.with_(T=12), 3, 3, 0, {"anchor_block": True}

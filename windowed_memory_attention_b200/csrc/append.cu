@@ -42,8 +42,10 @@ __device__ __forceinline__ int4 ld_stream(const int4* p) {
 #define GCA_APPEND_BLOCKS_PER_SM 8
 #endif
 
-// HSHIFT = log2(H) when H is a power of two (shifts instead of divisions), else -1
-template <int HSHIFT>
+// HSHIFT = log2(H) when H is a power of two (shifts instead of divisions), else -1;
+// ROPE: K is rotated by the 3D rotary encoding (a separate instantiation keeps
+// the plain copy's register count, and so its occupancy, unchanged)
+template <int HSHIFT, bool ROPE>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     const int lt = blockIdx.y;                 // layer-local index * 2 + tensor
     const int ll = lt >> 1;
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
                (long long)(slot0 + sl) * row_bytes + zc * 16;
     };
     // K with the 3D rotary encoding: each 16-byte chunk holds whole dim pairs
-    const bool rotate = tensor == 0 && p.rope.t != nullptr;
+    const bool rotate = ROPE && tensor == 0;
     auto rope_chunk = [&](int4& v, unsigned tok, unsigned chunk) {
         if (p.elem_bytes == 2) {
             uint32_t w[4] = {(uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w};
@@ -162,10 +164,12 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
                                  : ld_stream(reinterpret_cast<const int4*>(src) + u);
             }
         }
-        if (rotate) {
+        if constexpr (ROPE) {
+            if (rotate) {
 #pragma unroll
-            for (int i = 0; i < U; ++i)
-                if (dst[i] && !zero[i]) rope_chunk(val[i], tok[i], chunk[i]);
+                for (int i = 0; i < U; ++i)
+                    if (dst[i] && !zero[i]) rope_chunk(val[i], tok[i], chunk[i]);
+            }
         }
 #pragma unroll
         for (int i = 0; i < U; ++i)
@@ -186,14 +190,19 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     if (want < 1) want = 1;
     dim3 grid((unsigned)want, (unsigned)(2 * p.nlayers));
     const int hs = (p.H & (p.H - 1)) == 0 ? __builtin_ctz((unsigned)p.H) : -1;
+    if (p.rope.t) {
+        if (hs == 4) append_kernel<4, true><<<grid, 256, 0, s>>>(p);
+        else append_kernel<-1, true><<<grid, 256, 0, s>>>(p);
+        return cudaGetLastError();
+    }
     switch (hs) {
-        case 0: append_kernel<0><<<grid, 256, 0, s>>>(p); break;
-        case 1: append_kernel<1><<<grid, 256, 0, s>>>(p); break;
-        case 2: append_kernel<2><<<grid, 256, 0, s>>>(p); break;
-        case 3: append_kernel<3><<<grid, 256, 0, s>>>(p); break;
-        case 4: append_kernel<4><<<grid, 256, 0, s>>>(p); break;
-        case 5: append_kernel<5><<<grid, 256, 0, s>>>(p); break;
-        default: append_kernel<-1><<<grid, 256, 0, s>>>(p); break;
+        case 0: append_kernel<0, false><<<grid, 256, 0, s>>>(p); break;
+        case 1: append_kernel<1, false><<<grid, 256, 0, s>>>(p); break;
+        case 2: append_kernel<2, false><<<grid, 256, 0, s>>>(p); break;
+        case 3: append_kernel<3, false><<<grid, 256, 0, s>>>(p); break;
+        case 4: append_kernel<4, false><<<grid, 256, 0, s>>>(p); break;
+        case 5: append_kernel<5, false><<<grid, 256, 0, s>>>(p); break;
+        default: append_kernel<-1, false><<<grid, 256, 0, s>>>(p); break;
     }
     return cudaGetLastError();
 }

@@ -7,7 +7,7 @@
 // that may synchronise the device or take an unbounded time.  Such a caller
 // keeps the K/V pools in its own memory and calls gca_attend_pages_noalloc,
 // which launches the same tcgen05 attention kernel as gca_attend but puts its
-// split-KV partial results (and a device copy of the walk list) in one
+// split-KV partial results, their counters (and a device copy of the walk list) in one
 // file-scope __device__ array instead of cache-owned scratch.
 //
 // The array is gca_noalloc_scratch, kNoallocScratchBytes = 18 MiB, resident
@@ -20,6 +20,7 @@
 // read within one call).  Two calls whose GPU work overlaps (different
 // streams, or different devices' work is fine) race on the array.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/gca.h"
@@ -34,7 +35,9 @@ constexpr size_t kWalkBytes = (size_t)kNoallocMaxWalk * sizeof(int4);
 constexpr size_t kLseBytes = (size_t)kNoallocMaxSlots * 128 * sizeof(float);
 constexpr size_t kPartialBytes = (size_t)kNoallocMaxSlots * 128 * gca::kHeadDim * sizeof(float);
 constexpr size_t kStatusBytes = 256;
-constexpr size_t kNoallocScratchBytes = kStatusBytes + kWalkRawBytes + kWalkBytes + kLseBytes + kPartialBytes;
+constexpr size_t kCountBytes = (size_t)kNoallocMaxSlots * sizeof(unsigned long long);   // split-head counters
+constexpr size_t kNoallocScratchBytes =
+    kStatusBytes + kCountBytes + kWalkRawBytes + kWalkBytes + kLseBytes + kPartialBytes;
 static_assert(kNoallocScratchBytes <= (size_t)18 << 20, "scratch stays modest");
 
 }  // namespace
@@ -54,6 +57,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
 EncodeTiledFn g_encode = nullptr;
 AddressRangeFn g_range = nullptr;
+std::atomic<unsigned int> g_epoch{0};   // launch epochs of the split-head counters
 
 // Device address of the scratch array on the current device, looked up once
 // per device.
@@ -166,10 +170,12 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
         return GCA_ERR_INVALID_ARG;
     }
     int* d_status = reinterpret_cast<int*>(base);
-    gca_page_entry_t* walk_raw = reinterpret_cast<gca_page_entry_t*>(base + kStatusBytes);
-    int4* walk_dev = reinterpret_cast<int4*>(base + kStatusBytes + kWalkRawBytes);
-    float* ws_lse = reinterpret_cast<float*>(base + kStatusBytes + kWalkRawBytes + kWalkBytes);
-    float* ws_o = reinterpret_cast<float*>(base + kStatusBytes + kWalkRawBytes + kWalkBytes + kLseBytes);
+    unsigned long long* counts = reinterpret_cast<unsigned long long*>(base + kStatusBytes);
+    unsigned char* rest = base + kStatusBytes + kCountBytes;
+    gca_page_entry_t* walk_raw = reinterpret_cast<gca_page_entry_t*>(rest);
+    int4* walk_dev = reinterpret_cast<int4*>(rest + kWalkRawBytes);
+    float* ws_lse = reinterpret_cast<float*>(rest + kWalkRawBytes + kWalkBytes);
+    float* ws_o = reinterpret_cast<float*>(rest + kWalkRawBytes + kWalkBytes + kLseBytes);
 
     const gca_page_entry_t* src = walk;
     if (walk_on_host) {
@@ -221,11 +227,9 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     w = std::max<long long>(w, 1);
     p.seg = (int)((total + w - 1) / w);
     p.W = (int)((total + p.seg - 1) / p.seg);
-    bool need_merge = false;
-    for (int h = 0; h < num_heads && !need_merge; ++h)
-        need_merge = ((long long)h * nwalk) / p.seg != ((long long)(h + 1) * nwalk - 1) / p.seg;
+    p.merge_cnt = counts;
+    p.epoch = g_epoch.fetch_add(1) + 1;
     cudaError_t err = gca::launch_attend_sm100(tk, tv, p, st);
-    if (err == cudaSuccess && need_merge) err = gca::launch_merge(p, st);
     if (err != cudaSuccess) {
         cudaGetLastError();
         return GCA_ERR_CUDA;

@@ -14,35 +14,49 @@
 // segment read the same K/V pages in the same order at about the same time,
 // so each page comes from HBM once and from L2 for the others.  A segment that
 // covers a whole head writes the final output; heads split between segments
-// leave normalised partials plus their log-sum-exp for the merge kernel.
+// leave normalised partials plus their log-sum-exp, and the worker that
+// finishes a split head last (a per-(tile, head) counter) combines them.
 //
 // Per CTA (384 threads, one CTA per SM):
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread t owns query row t of
-//              its tile (TMEM lane t); loads Q into TMEM, reads S rows from
-//              TMEM, online softmax in the log2 domain, writes P (bf16) back
-//              over the S columns, final normalisation;
+//              its tile (TMEM lane t); writes its Q row into shared memory,
+//              reads S rows from TMEM, online softmax in the log2 domain,
+//              writes P (bf16) back over the S columns, final normalisation;
 //   warp 8     TMA producer: one (page, head) K tile and V tile per stage,
 //              128-byte swizzled boxes of P x 64 bf16, 4 stages;
-//   warp 9     MMA issuer (one thread) and TMEM owner (warps 10-11 idle).
-//              Per page j it issues
-//                S0 = Q0 K_j^T,  O1 += P1(j-1) V_{j-1},  S1 = Q1 K_j^T,
-//                O0 += P0(j) V_j
-//              so each softmax group overlaps the other group's two MMAs
-//              (A = Q or P from TMEM, B = K K-major / V MN-major from smem).
-// TMEM columns: S0, S1 (P aliased into their first P/2 columns), O0, O1, Q0,
-// Q1 — 448 of 512 for 128-token pages.  tcgen05 operations issued by one
-// thread execute in order, so S_t(j+1) is written only after PV_t(j) has read
-// P_t(j), and the commit after QK_t(j+1) also covers PV_t(j).
+//   warps 9/10 one MMA-issuing thread per tile (warp 9 also owns TMEM; warp
+//              11 idle).  Any wait in an issuing thread stalls its tcgen05.mma
+//              stream (the tensor core takes about one instruction ahead of
+//              the issuer): a mbarrier wait on an already completed phase
+//              costs ~200 cycles of tensor-pipe time.  With one issuer per
+//              tile, each issuer's waits are covered by the other's MMAs.
+//
+// Three rotating S buffers.  TMEM holds three S buffers of P columns and the
+// two tiles' O accumulators: 3 x 128 + 2 x 64 = 512 columns for 128-token
+// pages.  QK of tile t for page j (index i = 2j + t) writes buffer i % 3.  Per
+// page, tile t's issuer runs S_t(j) = Q_t K_j^T, then O_t += P_t(j-1) V_{j-1},
+// so each tile's next S is computed while its softmax of the current page
+// runs, and the two softmax groups work side by side instead of taking turns.
+// Buffer i % 3 last held index i - 3 (the other tile), whose PV reads its P:
+// the QK waits for that PV to complete (buf_free, one phase per use of the
+// buffer).  Q sits in shared memory (SS-form QK), two buffers per tile, so
+// the softmax warps load the next head's Q while the current head runs.
+//
+// A warp may start page j+1 (its S is ready) while the other warps of its
+// tile finish page j, so the "P written" barrier is split by page parity:
+// arrivals for page j+1 never count toward page j.
 //
 // Softmax: a page is exponentiated against the row's running max without
 // computing the page max first.  Since relative precision does not depend on
 // scale, values up to 2^64 are as good as values up to 1; a row whose page
 // sum reaches 2^64 (or overflows) takes the exact path instead: page max, O
-// rescaled by 2^(m_old - m_new), exponentials recomputed.  The first page of
-// every head always takes the exact path.  Scores are scaled and shifted with
-// packed f32x2 FMAs; two of every sixteen column pairs get 2^x from a
-// degree-3 minimax polynomial on the FMA pipe (exp2_poly_fit.py), the rest
-// from the MUFU unit (ex2.approx).
+// rescaled by 2^(m_old - m_new) once the previous PV has completed (the
+// page's K/V stage released by both tiles' PVs),
+// exponentials recomputed.  The first page of every head always takes the
+// exact path.  Scores are scaled and shifted with packed f32x2 FMAs; every
+// exponential runs on the MUFU unit (ex2.approx): with this schedule the
+// kernel is not MUFU-bound, and moving part of them to an FMA-pipe polynomial
+// measured slower.
 //
 // Every wait on an mbarrier is bounded by a %globaltimer deadline; on expiry
 // the thread raises the CTA abort flag and the device status word, every role
@@ -65,34 +79,18 @@ constexpr int kWarpMMA = 9;
 constexpr int kRegsSoftmax = 216;
 constexpr int kRegsProducer = 64;
 static_assert(256 * kRegsSoftmax + 128 * kRegsProducer <= kThreads * 168, "register split");
-#ifndef GCA_ATTEND_STAGES
-#define GCA_ATTEND_STAGES 4
-#endif
-#ifndef GCA_POLY_PAIRS
-#define GCA_POLY_PAIRS 2
-#endif
-constexpr int kStages = GCA_ATTEND_STAGES;
+constexpr int kStages = 4;
 constexpr int kRows = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
-constexpr int kPolyPairs = GCA_POLY_PAIRS;  // of each 16 column pairs, this many use the FMA-pipe 2^x
-
-// 2^f on [-1/2, 1/2], minimax relative error 7.5e-5 (exp2_poly_fit.py)
-constexpr float kExpC0 = 0x1.fff692p-1f;
-constexpr float kExpC1 = 0x1.62f31ap-1f;
-constexpr float kExpC2 = 0x1.f0de1ap-3f;
-constexpr float kExpC3 = 0x1.c3f76p-5f;
-
 template <int PAGE>
 struct Layout {
     static constexpr int kTileBytes = PAGE * 128;          // PAGE x 64 bf16
     static constexpr int kStageBytes = 2 * kTileBytes;     // K then V
-    static constexpr int kColS = 0;                        // + tile * PAGE (P in the first PAGE/2)
-    static constexpr int kColO = 2 * PAGE;                 // + tile * 64
-    static constexpr int kColQ = 2 * PAGE + 128;           // + tile * 32
-    static_assert(kColQ + 64 <= (int)kTmemCols, "TMEM budget");
-    static constexpr int kNumBars = 2 * kStages + 9;
-    static constexpr int kSmemBytes = kStages * kStageBytes + kNumBars * 8 + 16 + 1024;
+    static constexpr int kQBytes = 128 * 128;              // one tile's Q: 128 rows x 64 bf16, SW128
+    static_assert(3 * PAGE + 128 <= (int)kTmemCols, "TMEM budget: 3 S buffers + 2 O");
+    static constexpr int kNumBars = 2 * kStages + 27;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 4 * kQBytes + kNumBars * 8 + 16 + 1024;
 };
 
 // ---------------------------------------------------------------------------
@@ -121,6 +119,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -150,6 +149,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, b
         }
     }
 }
+
 
 __device__ __forceinline__ void fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -192,6 +192,16 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
         "r"(a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[smem desc] * B[smem desc]; descriptors as 32-bit halves
+__device__ __forceinline__ void mma_ss(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                       uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\n.reg .b64 ad, bd;\nsetp.ne.b32 p, %6, 0;\nmov.b64 ad, {%1, %2};\n"
+        "mov.b64 bd, {%3, %4};\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n}" ::"r"(d),
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // D[tmem] += A[tmem] * B[smem desc]; B given as its two 32-bit halves
 __device__ __forceinline__ void mma_ts_acc(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t b_hi,
                                            uint32_t idesc) {
@@ -221,13 +231,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
         : GCA_R8(0), GCA_R8(8), GCA_R8(16), GCA_R8(24)
         : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        GCA_W8(0), GCA_W8(8), GCA_W8(16), GCA_W8(24)
-        : "memory");
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : GCA_R8(0), GCA_R8(8)
+        : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
     asm volatile(
@@ -285,33 +294,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for two values on the FMA pipe: x = j + f, j = rne(x) through the
-// 1.5*2^23 shifter, p(f) by Horner, then j added to the exponent field.
-// x is clamped to >= -125 so the exponent never underflows into the sign;
-// an input below -125 (a masked key's -inf among them) gives exactly 0.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-    const bool z0 = x0 < -125.f, z1 = x1 < -125.f;
-    x0 = fmaxf(x0, -125.f);
-    x1 = fmaxf(x1, -125.f);
-    const uint64_t x = f2(x0, x1);
-    const uint64_t t = fadd2(x, f2(12582912.f, 12582912.f));
-    const uint64_t j = fadd2(t, f2(-12582912.f, -12582912.f));
-    const uint64_t f = ffma2(j, f2(-1.f, -1.f), x);
-    uint64_t p = ffma2(f2(kExpC3, kExpC3), f, f2(kExpC2, kExpC2));
-    p = ffma2(p, f, f2(kExpC1, kExpC1));
-    p = ffma2(p, f, f2(kExpC0, kExpC0));
-    float t0, t1, p0, p1;
-    unf2(t, t0, t1);
-    unf2(p, p0, p1);
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-    y0 = z0 ? 0.f : y0;
-    y1 = z1 ? 0.f : y1;
-}
 
 // ---------------------------------------------------------------------------
-// the kernel
 // ---------------------------------------------------------------------------
+// the kernel: two query tiles, three rotating S buffers
+// ---------------------------------------------------------------------------
+// QK_t(j) (tile t, page j) writes S buffer (2j + t) % 3.  The buffer's previous
+// user is QK of index 2j + t - 3, whose PV is issued before QK_t(j), so each
+// tile's next S is computed while its softmax of the current page runs.
 template <int PAGE>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -321,43 +311,66 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * L::kStageBytes);
+    const uint32_t qbase = sbase + kStages * L::kStageBytes;     // Q[t][buf] at + (2t+buf)*kQBytes
+    uint8_t* qsm = smem + kStages * L::kStageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + 4 * L::kQBytes);
     const uint32_t bar0 = smem_u32(bars);
     auto kv_full = [&](int s) { return bar0 + 8u * s; };
     auto kv_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto s_full = [&](int t) { return bar0 + 8u * (2 * kStages + t); };
-    auto p_full = [&](int t) { return bar0 + 8u * (2 * kStages + 2 + t); };
-    auto pv_done = [&](int t) { return bar0 + 8u * (2 * kStages + 4 + t); };
-    auto q_ready = [&](int t) { return bar0 + 8u * (2 * kStages + 6 + t); };
-    const uint32_t drain = bar0 + 8u * (2 * kStages + 8);
+    auto s_full = [&](int b) { return bar0 + 8u * (2 * kStages + b); };           // 3 buffers
+    // P of tile t written for page j: p_full(t, j & 1).  One barrier per page
+    // parity: a warp may start page j+1 (its S is already computed) while the
+    // tile's other warps still finish page j, so its arrivals must not count
+    // toward page j's phase; it cannot reach page j+2 before page j's phase
+    // completed (QK_t(j+2) is issued only after PV_t(j)).
+    auto p_full = [&](int t, int par) { return bar0 + 8u * (2 * kStages + 14 + 2 * t + par); };
+    auto q_ready = [&](int t, int b) { return bar0 + 8u * (2 * kStages + 7 + 2 * t + b); };
+    // drain(t): MMA thread t's last MMAs have completed (before TMEM is freed)
+    auto drain = [&](int t) { return bar0 + 8u * (2 * kStages + 18 + t); };
+    // buf_free(b): the PV that read S buffer b's P has completed, so the next
+    // QK may overwrite it (the two tiles' QKs and PVs come from two threads)
+    auto buf_free = [&](int b) { return bar0 + 8u * (2 * kStages + 20 + b); };
+    // o_done(t): PV_t of a head's last page has completed (one phase per head)
+    auto o_done = [&](int t) { return bar0 + 8u * (2 * kStages + 12 + t); };
+    // fused merge of a split head: every row of the tile has written its partial
+    // (mrg_all, 128 arrivals), then the tile's elected thread posts whether this
+    // CTA is the head's last worker (mrg_flag, 1 arrival)
+    auto mrg_all = [&](int t) { return bar0 + 8u * (2 * kStages + 23 + t); };
+    auto mrg_flag = [&](int t) { return bar0 + 8u * (2 * kStages + 25 + t); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);    // [2]: per tile
     const Ctl ctl{abort_flag, p.status};
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qp = blockIdx.x;                 // pair of 128-row query tiles
-    const int w = blockIdx.y;                  // worker (segment of the page stream)
+    const int qp = blockIdx.x;
+    const int w = blockIdx.y;
     const long long total = (long long)p.H * p.nwalk;
     const long long g0 = (long long)w * p.seg;
     const long long g1 = (g0 + p.seg < total) ? g0 + p.seg : total;
     const int J = (int)(g1 - g0);
-    // (head, entry) of the first page; every role then steps them incrementally
     const int h_start = (int)(g0 / p.nwalk);
     const int e_start = (int)(g0 - (long long)h_start * p.nwalk);
+    const int h_last = (int)((g1 - 1) / p.nwalk);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(kv_full(s), 1);
-            mbar_init(kv_empty(s), 1);
+            mbar_init(kv_empty(s), 2);          // both tiles' PV of the stage's page
         }
+        for (int b = 0; b < 3; ++b) mbar_init(s_full(b), 1);
         for (int t = 0; t < 2; ++t) {
-            mbar_init(s_full(t), 1);
-            mbar_init(p_full(t), kRows);
-            mbar_init(pv_done(t), 1);
-            mbar_init(q_ready(t), kRows);
+            mbar_init(p_full(t, 0), kRows);
+            mbar_init(p_full(t, 1), kRows);
+            mbar_init(q_ready(t, 0), kRows);
+            mbar_init(q_ready(t, 1), kRows);
+            mbar_init(o_done(t), 1);
+            mbar_init(mrg_all(t), kRows);
+            mbar_init(mrg_flag(t), 1);
         }
-        mbar_init(drain, 1);
+        for (int t = 0; t < 2; ++t) mbar_init(drain(t), 1);
+        for (int b = 0; b < 3; ++b) mbar_init(buf_free(b), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -410,104 +423,103 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 }
             }
             if (!ok) {
-                // let every load already issued land before the CTA exits
                 const int from = issued > kStages ? issued - kStages : 0;
                 for (int j = from; j < issued; ++j)
                     wait_bar(kv_full(j % kStages), (j / kStages) & 1, ctl, false);
             }
         }
         __syncwarp();
-    } else if (warp == kWarpMMA) {
-        // ------------------------------------------------------------ MMA issuer
+      } else if (warp == kWarpMMA || warp == kWarpMMA + 1) {
+        // ------------------------------------------------------------ MMA issuers
+        // one thread per query tile: warp 9 issues tile 0's MMAs, warp 10 tile
+        // 1's, so one thread's waits are covered by the other's MMAs
         if (lane == 0) {
+            const int t = warp - kWarpMMA;
             constexpr uint32_t kIdescQK = idesc_bf16(kRows, PAGE, false);
             constexpr uint32_t kIdescPV = idesc_bf16(kRows, 64, true);
-            // descriptors of stage 0; stage s and step kk add constants to the
-            // start-address field (16-byte units): K steps 32 bytes, V steps 2 KB
             const uint64_t kdesc0 = desc_sw128(sbase, 16, 1024);
             const uint64_t vdesc0 = desc_sw128(sbase + L::kTileBytes, L::kTileBytes, 1024);
-            constexpr uint64_t kStageStep = L::kStageBytes >> 4;
-            // descriptor halves: only the low word (start address) varies
+            const uint64_t qdesc0 = desc_sw128(qbase, 16, 1024);
+            constexpr uint32_t kStageStep = L::kStageBytes >> 4;
+            constexpr uint32_t kQStep = L::kQBytes >> 4;
             const uint32_t kd_lo0 = (uint32_t)kdesc0, kd_hi = (uint32_t)(kdesc0 >> 32);
             const uint32_t vd_lo0 = (uint32_t)vdesc0, vd_hi = (uint32_t)(vdesc0 >> 32);
-            auto qk = [&](int t, int st) {
-                const uint64_t kd = kdesc0 + st * kStageStep;
-                const uint32_t kd_lo = kd_lo0 + st * (uint32_t)kStageStep;
-                const uint32_t scol = tmem + L::kColS + t * PAGE;
-                const uint32_t qcol = tmem + L::kColQ + t * 32;
-                mma_ts(scol, qcol, kd, kIdescQK, 0u);
-#pragma unroll
-                for (int kk = 1; kk < 4; ++kk)   // 16 head dims per step
-                    mma_ts_acc(scol, qcol + kk * 8, kd_lo + 2 * kk, kd_hi, kIdescQK);
-                mma_commit(s_full(t));
-            };
-            // pv_done is only needed at the end of a head: the commit after the
-            // next QK_t covers PV_t for the softmax
-            auto pv = [&](int t, int j, int st, bool first, bool last) -> bool {
-                if (!wait_bar(p_full(t), j & 1, ctl)) return false;
-                fence_after();
-                const uint64_t vd = vdesc0 + st * kStageStep;
-                const uint32_t vd_lo = vd_lo0 + st * (uint32_t)kStageStep;
-                const uint32_t ocol = tmem + L::kColO + t * 64;
-                const uint32_t pcol = tmem + L::kColS + t * PAGE;
-                mma_ts(ocol, pcol, vd, kIdescPV, first ? 0u : 1u);
-#pragma unroll
-                for (int kk = 1; kk < PAGE / 16; ++kk)   // 16 keys per step
-                    mma_ts_acc(ocol, pcol + kk * 8, vd_lo + 128 * kk, vd_hi, kIdescPV);
-                if (last) mma_commit(pv_done(t));
-                if (t == 1) mma_commit(kv_empty(st));
-                return true;
-            };
+            const uint32_t qd_lo0 = (uint32_t)qdesc0 + 2 * t * kQStep, qd_hi = (uint32_t)(qdesc0 >> 32);
+            const uint32_t ocol = tmem + 3 * PAGE + t * 64;
             bool ok = true;
-            int sidx = 0;
+            int hs = 0;                                  // heads started in this segment
             int e = e_start;
             bool prev_first = false, prev_last = false;
             int st = 0, prev_st = 0;
-            for (int j = 0; j < J; ++j) {
-                const bool seg_first = (j == 0) || (e == 0);
-                const bool seg_last = (j == J - 1) || (e == p.nwalk - 1);
-                if (seg_first && !wait_bar(q_ready(0), sidx & 1, ctl)) { ok = false; break; }
-                if (!wait_bar(kv_full(st), (j / kStages) & 1, ctl)) { ok = false; break; }
-                fence_after();
-                qk(0, st);
-                if (j > 0 && !pv(1, j - 1, prev_st, prev_first, prev_last)) { ok = false; break; }
-                if (seg_first) {
-                    if (!wait_bar(q_ready(1), sidx & 1, ctl)) { ok = false; break; }
-                    ++sidx;
+            for (int j = 0; j <= J && ok; ++j) {
+                const bool live = j < J;
+                const bool seg_first = live && ((j == 0) || (e == 0));
+                const bool seg_last = live && ((j == J - 1) || (e == p.nwalk - 1));
+                if (live) {
+                    const int qb = seg_first ? (hs & 1) : ((hs - 1) & 1);
+                    if (seg_first) {
+                        if (!wait_bar(q_ready(t, hs & 1), (hs >> 1) & 1, ctl)) { ok = false; break; }
+                        ++hs;
+                    }
+                    if (!wait_bar(kv_full(st), (j / kStages) & 1, ctl)) { ok = false; break; }
+                    // S buffer i % 3 (i = 2j + t) was last read, as P, by the PV of index i - 3
+                    const int i = 2 * j + t;
+                    const int b = i % 3;
+                    if (i >= 3 && !wait_bar(buf_free(b), ((i / 3) - 1) & 1, ctl)) { ok = false; break; }
                     fence_after();
+                    const uint32_t kd_lo = kd_lo0 + st * kStageStep;
+                    const uint32_t qd_lo = qd_lo0 + qb * kQStep;
+                    const uint32_t scol = tmem + b * PAGE;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // 16 head dims per step: +32 bytes
+                        mma_ss(scol, qd_lo + 2 * kk, qd_hi, kd_lo + 2 * kk, kd_hi, kIdescQK, kk ? 1u : 0u);
+                    mma_commit(s_full(b));
                 }
-                qk(1, st);
-                if (!pv(0, j, st, seg_first, seg_last)) { ok = false; break; }
+                if (j > 0) {
+                    // O_t += P_t(j-1) V_{j-1} once the tile's softmax has written P
+                    const int jj = j - 1;
+                    if (!wait_bar(p_full(t, jj & 1), (jj >> 1) & 1, ctl)) { ok = false; break; }
+                    fence_after();
+                    const int b = (2 * jj + t) % 3;
+                    const uint64_t vd = vdesc0 + prev_st * kStageStep;
+                    const uint32_t vd_lo = vd_lo0 + prev_st * kStageStep;
+                    const uint32_t pcol = tmem + b * PAGE;
+                    mma_ts(ocol, pcol, vd, kIdescPV, prev_first ? 0u : 1u);
+#pragma unroll
+                    for (int kk = 1; kk < PAGE / 16; ++kk)   // 16 keys per step
+                        mma_ts_acc(ocol, pcol + kk * 8, vd_lo + 128 * kk, vd_hi, kIdescPV);
+                    mma_commit(buf_free(b));
+                    if (prev_last) mma_commit(o_done(t));
+                    mma_commit(kv_empty(prev_st));
+                }
                 prev_first = seg_first;
                 prev_last = seg_last;
                 prev_st = st;
                 st = (st + 1 == kStages) ? 0 : st + 1;
                 if (++e == p.nwalk) e = 0;
             }
-            if (ok) pv(1, J - 1, prev_st, prev_first, prev_last);
-            // drain: every MMA issued above completes before TMEM is released
-            mma_commit(drain);
-            wait_bar(drain, 0, ctl, false);
+            // drain: every MMA this thread issued completes before TMEM is released
+            mma_commit(drain(t));
+            wait_bar(drain(t), 0, ctl, false);
         }
         __syncwarp();
       }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ------------------------------------------------------------ softmax
-        const int t = warp >> 2;                       // query tile of this warp group
+        const int t = warp >> 2;
         const int quarter = warp & 3;
-        const int rl = quarter * 32 + lane;            // row in the tile, TMEM lane
+        const int rl = quarter * 32 + lane;
         const int row = (qp * 2 + t) * kRows + rl;
         const bool valid = row < p.R;
         const int qframe = p.first_query_frame + (valid ? row / p.Lq : 0);
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t t_s = tmem + lane_base + L::kColS + t * PAGE;
-        const uint32_t t_o = tmem + lane_base + L::kColO + t * 64;
-        const uint32_t t_q = tmem + lane_base + L::kColQ + t * 32;
+        const uint32_t t_o = tmem + lane_base + 3 * PAGE + t * 64;
         const float sl2 = p.scale_log2;
         const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
 
-        auto load_q = [&](int h) {
+        // Q of head h into Q buffer qb of this tile (K-major, 128-byte swizzle)
+        auto load_q = [&](int h, int qb) {
             uint32_t r[32];
             if (valid) {
                 const uint4* src = reinterpret_cast<const uint4*>(qg + ((long long)row * p.H + h) * 64);
@@ -520,8 +532,6 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     r[4 * i + 3] = v.w;
                 }
                 if (p.rope.t) {
-                    // 3D rotary encoding at the row's (frame, token) position:
-                    // each 32-bit word holds dim pair i in fp32, rounded back to bf16
                     const int u = row % p.Lq;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -535,17 +545,21 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 #pragma unroll
                 for (int i = 0; i < 32; ++i) r[i] = 0u;
             }
-            tmem_st32(t_q, r);
-            tmem_wait_st();
-            fence_before();
-            mbar_arrive(q_ready(t));
+            uint8_t* qrow = qsm + (2 * t + qb) * L::kQBytes + rl * 128;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<uint4*>(qrow + ((i ^ (rl & 7)) * 16)) =
+                    make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(q_ready(t, qb));
         };
         auto all_ok = [&](bool ok) { return __all_sync(0xffffffffu, ok); };
 
         float m_run = -INFINITY, l_run = 0.f;
-        int segs_done = 0;                             // pv_done(t) phases consumed
-        load_q(h_start);
-        // walk entries are read one page ahead, off the critical path
+        int hs = 0;                                    // heads started
+        int hd = 0;                                    // heads finished (o_done phases)
+        int mg = 0;                                    // fused merges done (mrg_all / mrg_flag phases)
+        load_q(h_start, 0);
         int4 ent_next = __ldg(&p.walk[e_start]);
         int h = h_start, e = e_start - 1;
         for (int j = 0; j < J; ++j) {
@@ -558,13 +572,18 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             if (seg_first) {
                 m_run = -INFINITY;
                 l_run = 0.f;
+                // the next head's Q goes to the other buffer while this head runs;
+                // that buffer's last reader (the previous head's QKs) has completed
+                if (h < h_last) load_q(h + 1, (hs + 1) & 1);
+                ++hs;
             }
             const int4 ent = ent_next;
             if (j + 1 < J) ent_next = __ldg(&p.walk[e + 1 == p.nwalk ? 0 : e + 1]);
             const int nvis = visible_prefix(p.rule, ent, qframe);
+            const int b = (2 * j + t) % 3;
+            const uint32_t t_s = tmem + lane_base + b * PAGE;
 
-            // S_t(j) is complete, and so is PV_t(j-1) (one commit covers both)
-            if (!all_ok(wait_bar(s_full(t), j & 1, ctl))) break;
+            if (!all_ok(wait_bar(s_full(b), ((2 * j + t) / 3) & 1, ctl))) break;
             fence_after();
             uint32_t r[PAGE];
             auto load_s = [&]() {
@@ -576,7 +595,6 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     for (int c = 0; c < PAGE; ++c) r[c] = (c < nvis) ? r[c] : 0xff800000u;
                 }
             };
-            // r <- 2^(s * scale_log2 - msub) in place; returns the row sum
             auto exps = [&](float msub) -> float {
                 const uint64_t sl2v = f2(sl2, sl2);
                 const uint64_t nmv = f2(-msub, -msub);
@@ -586,12 +604,8 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     const uint64_t x = ffma2(f2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nmv);
                     float x0, x1, p0, p1;
                     unf2(x, x0, x1);
-                    if (((c >> 1) & 15) < kPolyPairs) {
-                        exp2_poly2(x0, x1, p0, p1);
-                    } else {
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                    }
+                    p0 = ex2(x0);
+                    p1 = ex2(x1);
                     rs2[(c >> 1) & 3] = fadd2(rs2[(c >> 1) & 3], f2(p0, p1));
                     r[c] = __float_as_uint(p0);
                     r[c + 1] = __float_as_uint(p1);
@@ -605,10 +619,6 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             };
             load_s();
 
-            // Fast path: exponentiate against the running max without looking
-            // for this page's max.  Values up to 2^64 are exact enough (relative
-            // precision does not depend on scale) and far from overflow; a row
-            // whose page sum reaches 2^64 (or inf / NaN) takes the exact path.
             float alpha = 1.f;
             bool resc = false;
             bool fast = m_run != -INFINITY;
@@ -618,10 +628,7 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 fast = rs < 0x1p64f;
             }
             if (!__all_sync(0xffffffffu, fast)) {
-                // r was overwritten by a fast attempt in some lanes; the reload is
-                // warp-collective, so every lane of the warp takes it
                 if (__any_sync(0xffffffffu, m_run != -INFINITY)) load_s();
-                // exact row max: 16 independent three-input max chains, then a tree
                 float acc[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(r[i]);
@@ -649,25 +656,28 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             }
 
             if (__any_sync(0xffffffffu, resc)) {
-                // PV_t(j-1) has completed (covered by the s_full commit)
+                // O_t holds PV_t up to page j-1 once that PV has completed
+                // both tiles' PVs of page j-1 have completed once its K/V stage is released
+                if (!all_ok(wait_bar(kv_empty((j - 1) % kStages), ((j - 1) / kStages) & 1, ctl))) break;
+                fence_after();
                 const uint64_t a2v = f2(alpha, alpha);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t o[32];
-                    tmem_ld32(t_o + 32 * half, o);
+#pragma unroll 1
+                for (int part = 0; part < 4; ++part) {
+                    uint32_t o[16];
+                    tmem_ld16(t_o + 16 * part, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int d = 0; d < 32; d += 2) {
+                    for (int d = 0; d < 16; d += 2) {
                         float x0, x1;
                         unf2(fmul2(f2(__uint_as_float(o[d]), __uint_as_float(o[d + 1])), a2v), x0, x1);
                         o[d] = __float_as_uint(x0);
                         o[d + 1] = __float_as_uint(x1);
                     }
-                    tmem_st32(t_o + 32 * half, o);
+                    tmem_st16(t_o + 16 * part, o);
                 }
             }
 
-            // P (bf16) written over the S columns
+            // P (bf16) over the first PAGE/2 columns of the page's S buffer
 #pragma unroll
             for (int c = 0; c < PAGE / 32; ++c) {
                 uint32_t pk[16];
@@ -679,11 +689,12 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             l_run = l_run * alpha + rs;
             tmem_wait_st();
             fence_before();
-            mbar_arrive(p_full(t));
+            mbar_arrive(p_full(t, j & 1));
 
             if (seg_last) {
-                if (!all_ok(wait_bar(pv_done(t), segs_done & 1, ctl))) break;
-                ++segs_done;
+                // the head's last PV_t has completed -> O_t final for this head
+                if (!all_ok(wait_bar(o_done(t), hd & 1, ctl))) break;
+                ++hd;
                 fence_after();
                 uint32_t o[64];
                 tmem_ld32(t_o, o);
@@ -708,16 +719,78 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         }
                         if (p.lse) p.lse[(long long)row * p.H + h] = lse2 * 0.69314718055994531f;
                     }
-                } else if (valid) {
-                    const long long slot = (long long)(qp * 2 + t) * (p.W + p.H - 1) + w + h;
-                    float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kRows + rl) * 64);
+                } else {
+                    // the head is split between workers: leave this worker's
+                    // normalised partial and log2-sum-exp; the worker that
+                    // finishes the head last combines all of them
+                    const long long base = (long long)(qp * 2 + t) * (p.W + p.H - 1) + h;
+                    if (valid) {
+                        const long long slot = base + w;
+                        float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kRows + rl) * 64);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[4 * i + 0]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                             __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-                    p.ws_lse[slot * kRows + rl] = lse2;
+                        for (int i = 0; i < 16; ++i)
+                            dst[i] = make_float4(__uint_as_float(o[4 * i + 0]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                                 __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+                        p.ws_lse[slot * kRows + rl] = lse2;
+                    }
+                    __threadfence();
+                    mbar_arrive(mrg_all(t));
+                    if (!all_ok(wait_bar(mrg_all(t), mg & 1, ctl))) break;
+                    if (rl == 0) {
+                        // count the head's finished workers in this launch: the
+                        // counter's high word is the launch epoch, the low word
+                        // the count, so no reset between launches is needed
+                        unsigned long long* cnt = p.merge_cnt + (long long)(qp * 2 + t) * p.H + h;
+                        unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt), nxt;
+                        for (;;) {
+                            nxt = ((unsigned long long)p.epoch << 32) |
+                                  ((unsigned)(cur >> 32) == p.epoch ? (cur & 0xffffffffull) + 1 : 1ull);
+                            const unsigned long long seen = atomicCAS(cnt, cur, nxt);
+                            if (seen == cur) break;
+                            cur = seen;
+                        }
+                        last_flag[t] = (int)(nxt & 0xffffffffull) == w_hi - w_lo + 1;
+                        mbar_arrive(mrg_flag(t));
+                    }
+                    if (!all_ok(wait_bar(mrg_flag(t), mg & 1, ctl))) break;
+                    ++mg;
+                    if (last_flag[t] && valid) {
+                        __threadfence();
+                        float mx = -INFINITY;
+                        for (int ww = w_lo; ww <= w_hi; ++ww)
+                            mx = fmaxf(mx, __ldcg(p.ws_lse + (base + ww) * kRows + rl));
+                        float acc[64];
+#pragma unroll
+                        for (int d = 0; d < 64; ++d) acc[d] = 0.f;
+                        float den = 0.f;
+                        for (int ww = w_lo; ww <= w_hi; ++ww) {
+                            const float l2 = __ldcg(p.ws_lse + (base + ww) * kRows + rl);
+                            if (l2 == -INFINITY) continue;
+                            const float wt = ex2(l2 - mx);
+                            den += wt;
+                            const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((base + ww) * kRows + rl) * 64);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float4 v = __ldcg(src + i);
+                                acc[4 * i + 0] = fmaf(wt, v.x, acc[4 * i + 0]);
+                                acc[4 * i + 1] = fmaf(wt, v.y, acc[4 * i + 1]);
+                                acc[4 * i + 2] = fmaf(wt, v.z, acc[4 * i + 2]);
+                                acc[4 * i + 3] = fmaf(wt, v.w, acc[4 * i + 3]);
+                            }
+                        }
+                        const float dinv = den > 0.f ? 1.f / den : 0.f;
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                              ((long long)row * p.H + h) * 64);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_uint4(pack_bf16(acc[8 * i + 0] * dinv, acc[8 * i + 1] * dinv),
+                                                pack_bf16(acc[8 * i + 2] * dinv, acc[8 * i + 3] * dinv),
+                                                pack_bf16(acc[8 * i + 4] * dinv, acc[8 * i + 5] * dinv),
+                                                pack_bf16(acc[8 * i + 6] * dinv, acc[8 * i + 7] * dinv));
+                        if (p.lse)
+                            p.lse[(long long)row * p.H + h] = (den > 0.f ? mx + __log2f(den) : -INFINITY) * 0.69314718055994531f;
+                    }
                 }
-                if (j < J - 1) load_q(h + 1);
             }
         }
     }
@@ -747,52 +820,6 @@ __global__ void bounded_wait_selftest(int* status, unsigned long long timeout_ns
     wait_bar(smem_u32(&bar), 0, ctl, true, timeout_ns);
 }
 
-// Combine the partials of heads that were split between workers.
-__global__ void __launch_bounds__(128) merge_kernel(const AttendParams p) {
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long long)p.R * p.H) return;
-    const int row = (int)(idx / p.H);
-    const int h = (int)(idx - (long long)row * p.H);
-    const int w_lo = (int)(((long long)h * p.nwalk) / p.seg);
-    const int w_hi = (int)(((long long)(h + 1) * p.nwalk - 1) / p.seg);
-    if (w_lo == w_hi) return;
-    const int qt = row / kRows, rl = row % kRows;
-    const long long base = (long long)qt * (p.W + p.H - 1) + h;
-    float mx = -INFINITY;
-    for (int w = w_lo; w <= w_hi; ++w) mx = fmaxf(mx, p.ws_lse[(base + w) * kRows + rl]);
-    float acc[64];
-#pragma unroll
-    for (int d = 0; d < 64; ++d) acc[d] = 0.f;
-    float den = 0.f;
-    for (int w = w_lo; w <= w_hi; ++w) {
-        const float l2 = p.ws_lse[(base + w) * kRows + rl];
-        if (l2 == -INFINITY) continue;
-        const float wt = exp2f(l2 - mx);
-        den += wt;
-        const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((base + w) * kRows + rl) * 64);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 v = src[i];
-            acc[4 * i + 0] += wt * v.x;
-            acc[4 * i + 1] += wt * v.y;
-            acc[4 * i + 2] += wt * v.z;
-            acc[4 * i + 3] += wt * v.w;
-        }
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((long long)row * p.H + h) * 64);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint4 v;
-        v.x = pack_bf16(acc[8 * i + 0] * inv, acc[8 * i + 1] * inv);
-        v.y = pack_bf16(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv);
-        v.z = pack_bf16(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv);
-        v.w = pack_bf16(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv);
-        dst[i] = v;
-    }
-    if (p.lse) p.lse[(long long)row * p.H + h] = (mx + log2f(den)) * 0.69314718055994531f;
-}
-
 template <int PAGE>
 cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const AttendParams& p,
                         cudaStream_t s) {
@@ -819,10 +846,5 @@ cudaError_t launch_bounded_wait_selftest(int* status, unsigned long long timeout
     return cudaGetLastError();
 }
 
-cudaError_t launch_merge(const AttendParams& p, cudaStream_t s) {
-    const long long n = (long long)p.R * p.H;
-    merge_kernel<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(p);
-    return cudaGetLastError();
-}
 
 }  // namespace gca

@@ -93,13 +93,16 @@ struct gca_cache {
     int tup_n = 0;
     float* ws_o = nullptr;
     float* ws_lse = nullptr;
+    unsigned long long* merge_cnt = nullptr;   // [QT_max][H] split-head counters
+    unsigned int epoch = 0;                    // launches of the bf16 kernel
     size_t ws_slots = 0;
     int* h_status = nullptr;
     int* d_status = nullptr;
     // staging for host-memory arguments: inputs are copied on the library's own
     // copy stream (so uploads overlap the caller's compute stream), guarded by
     // events; pinned host outputs are written by the kernels directly
-    cudaStream_t copy = nullptr;
+    cudaStream_t copy = nullptr;      // query-block uploads (ring of staging slots)
+    cudaStream_t copy_kv = nullptr;   // K/V uploads, so they never queue behind the ring
     void* st_k = nullptr;
     void* st_v = nullptr;
     cudaEvent_t kv_free = nullptr, kv_ready = nullptr;
@@ -137,6 +140,7 @@ void release(gca_cache* c) {
     cudaFree(c->d_walk_f);
     cudaFree(c->ws_o);
     cudaFree(c->ws_lse);
+    cudaFree(c->merge_cnt);
     cudaFree(c->st_k);
     cudaFree(c->st_v);
     for (int i = 0; i < kQRing; ++i) {
@@ -151,6 +155,7 @@ void release(gca_cache* c) {
     if (c->kv_free) cudaEventDestroy(c->kv_free);
     if (c->kv_ready) cudaEventDestroy(c->kv_ready);
     if (c->copy) cudaStreamDestroy(c->copy);
+    if (c->copy_kv) cudaStreamDestroy(c->copy_kv);
     for (int i = 0; i < kRing; ++i) {
         if (c->h_stage[i]) cudaFreeHost(c->h_stage[i]);
         if (c->stage_ev[i]) cudaEventDestroy(c->stage_ev[i]);
@@ -203,7 +208,7 @@ Mem classify(const void* ptr, void** alias = nullptr) {
 
 bool is_device_ptr(const void* ptr) { return classify(ptr) == Mem::kDevice; }
 
-// Upload a host input into a staging buffer on the cache's copy stream: the
+// Upload a host query block into a staging slot on the cache's copy stream: the
 // copy waits until the buffer's previous reader (on the caller's stream) is
 // done (`free_ev`), and the caller's stream waits for the copy (`ready_ev`).
 // The caller records free_ev on its stream after the kernel that reads dst.
@@ -222,16 +227,16 @@ bool stage_kv(gca_cache* c, const void* k, const void* v, size_t bytes, cudaStre
     *vd = v;
     const bool kh = !is_device_ptr(k), vh = !is_device_ptr(v);
     if (!kh && !vh) return true;
-    if (cudaStreamWaitEvent(c->copy, c->kv_free, 0) != cudaSuccess) return false;
+    if (cudaStreamWaitEvent(c->copy_kv, c->kv_free, 0) != cudaSuccess) return false;
     if (kh) {
-        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, c->copy) != cudaSuccess) return false;
+        if (cudaMemcpyAsync(c->st_k, k, bytes, cudaMemcpyHostToDevice, c->copy_kv) != cudaSuccess) return false;
         *kd = c->st_k;
     }
     if (vh) {
-        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, c->copy) != cudaSuccess) return false;
+        if (cudaMemcpyAsync(c->st_v, v, bytes, cudaMemcpyHostToDevice, c->copy_kv) != cudaSuccess) return false;
         *vd = c->st_v;
     }
-    return cudaEventRecord(c->kv_ready, c->copy) == cudaSuccess &&
+    return cudaEventRecord(c->kv_ready, c->copy_kv) == cudaSuccess &&
            cudaStreamWaitEvent(st, c->kv_ready, 0) == cudaSuccess;
 }
 
@@ -386,15 +391,10 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
         w = std::max<long long>(w, 1);
         p.seg = ceil_div(total, w);
         p.W = ceil_div(total, p.seg);
-        bool need_merge = false;
-        for (int h = 0; h < g.num_heads && !need_merge; ++h)
-            need_merge = ((long long)h * p.nwalk) / p.seg != ((long long)(h + 1) * p.nwalk - 1) / p.seg;
+        p.merge_cnt = c->merge_cnt;
+        p.epoch = ++c->epoch;
         err = gca::launch_attend_sm100(c->tmK, c->tmV, p, st);
         c->launches += 1;
-        if (err == cudaSuccess && need_merge) {
-            err = gca::launch_merge(p, st);
-            c->launches += 1;
-        }
     } else {
         p.QT = ceil_div(R, kTileRows);
         p.W = 1;
@@ -548,8 +548,11 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     const int qp_max = (qt_max + 1) / 2;
     c->ws_slots = 2 * (size_t)std::max(c->sms, qp_max) + (size_t)qt_max * (g.num_heads - 1);
     if (g.dtype == GCA_DTYPE_BF16) {
+        const size_t cnt_bytes = (size_t)qt_max * g.num_heads * sizeof(unsigned long long);
         ok = ok && cudaMalloc(&c->ws_o, c->ws_slots * kTileRows * gca::kHeadDim * sizeof(float)) == cudaSuccess &&
-             cudaMalloc(&c->ws_lse, c->ws_slots * kTileRows * sizeof(float)) == cudaSuccess;
+             cudaMalloc(&c->ws_lse, c->ws_slots * kTileRows * sizeof(float)) == cudaSuccess &&
+             cudaMalloc(&c->merge_cnt, cnt_bytes) == cudaSuccess &&
+             cudaMemset(c->merge_cnt, 0, cnt_bytes) == cudaSuccess;
     }
     ok = ok && cudaHostAlloc((void**)&c->h_status, sizeof(int), cudaHostAllocMapped) == cudaSuccess;
     if (ok) {
@@ -558,6 +561,7 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
     }
     const size_t frame_bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
     ok = ok && cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&c->copy_kv, cudaStreamNonBlocking) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->kv_free, cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->kv_ready, cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; ok && i < kQRing; ++i)

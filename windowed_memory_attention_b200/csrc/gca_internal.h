@@ -102,13 +102,16 @@ struct AttendParams {
     float* ws_lse;            // [QT*(W+H-1)][128] partial log2-sum-exp
     int* status;              // device status word (host-mapped)
     RopeTables rope;          // q rotated on load when rope.t is set
+    // split heads: per-(query tile, head) count of finished workers, tagged
+    // with the launch's epoch in the high word (no reset between launches)
+    unsigned long long* merge_cnt;   // [QT][H]
+    unsigned int epoch;
 };
 
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
                                 const AttendParams& p, cudaStream_t s);
-cudaError_t launch_merge(const AttendParams& p, cudaStream_t s);
 cudaError_t launch_bounded_wait_selftest(int* status, unsigned long long timeout_ns, cudaStream_t s);
 cudaError_t launch_attend_f32(const AttendParams& p, const void* kpool, const void* vpool,
                               cudaStream_t s);
