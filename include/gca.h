@@ -19,10 +19,21 @@
  * device copy of the walk list.  Caller-owned: every pointer passed to a call.
  *
  * Pointers: q, k, v, out and lse may be device pointers or host pointers
- * (pinned or pageable).  Host inputs are staged through library buffers with
- * cudaMemcpyAsync on the given stream; host outputs are filled by an async
- * copy on that stream, so the caller synchronises the stream before reading
- * them.  Device pointers must stay valid until the stream has consumed them.
+ * (pinned or pageable).  Host inputs are staged through library device
+ * buffers by cudaMemcpyAsync on library copy streams; host outputs are written
+ * to library device buffers and copied back the same way.  The stream argument
+ * waits for those copies, so the caller synchronises the stream before
+ * reading a host output.  Device pointers must stay valid until the stream has
+ * consumed them.
+ *
+ * A call whose pointer arguments are ALL in host memory does not wait for
+ * earlier work on the stream: its kernels follow the cache's earlier calls
+ * only, on a library stream, so one call's copy back overlaps the next call's
+ * kernels (the stream still waits for the call).  Its host inputs are read
+ * after the call is made: the caller fills them before the call (not with
+ * work queued on the stream) and leaves them unchanged until the stream has
+ * completed the call.  Any other call (at least one device pointer) runs in
+ * the stream's order.
  *
  * Streams: every GPU step is asynchronous on the stream argument (a
  * cudaStream_t; NULL = legacy default stream).  Calls on one cache must be

@@ -188,6 +188,48 @@ def test_host_pointer_path_matches_device_path():
         assert torch.equal(lse_d.cpu(), lse_h)
 
 
+def test_all_host_calls_on_a_side_stream_match_device_path():
+    """Calls whose pointers are all host memory run on the library's stream and
+    overlap their copies back; the caller's stream still waits for each call,
+    so synchronising that stream alone makes the outputs readable.  Device-
+    pointer calls interleaved with them keep the cache's order."""
+    w = inputs.TINY_BF16.with_(L=3)
+    a = gca.Cache.for_workload(w)
+    b = gca.Cache.for_workload(w)
+    side = torch.cuda.Stream()
+    for t in range(14):
+        k, v, q = (inputs.draw(w, t, x) for x in "kvq")
+        a.append(k.cuda(), v.cuda())
+        a.evict()
+        mixed = t % 5 == 3            # every fifth frame goes through device pointers
+        with torch.cuda.stream(side):
+            if mixed:
+                b.append(k.cuda(), v.cuda(), stream=side)
+            else:
+                b.append(k.pin_memory(), v.pin_memory(), stream=side)
+        b.evict()
+        outs_d = [attend(a, l, q[l:l + 1].cuda()) for l in range(w.L)]
+        torch.cuda.synchronize()
+        q_h = q.pin_memory()
+        out_h = [torch.empty_like(q[0:1]).pin_memory() for _ in range(w.L)]
+        lse_h = [torch.empty(q[0:1].shape[:3], dtype=torch.float32).pin_memory() for _ in range(w.L)]
+        for l in range(w.L):
+            if mixed and l == 1:
+                o_dev = torch.empty_like(q[0:1], device="cuda")
+                l_dev = torch.empty(q[0:1].shape[:3], dtype=torch.float32, device="cuda")
+                b.attend(l, q_h[l:l + 1], o_dev, l_dev, stream=side)
+                with torch.cuda.stream(side):
+                    out_h[l].copy_(o_dev, non_blocking=True)
+                    lse_h[l].copy_(l_dev, non_blocking=True)
+            else:
+                b.attend(l, q_h[l:l + 1], out_h[l], lse_h[l], stream=side)
+        side.synchronize()
+        for l in range(w.L):
+            assert torch.equal(outs_d[l][0].cpu(), out_h[l]), (t, l)
+            assert torch.equal(outs_d[l][1].cpu(), lse_h[l]), (t, l)
+    assert b.status() == 0
+
+
 def test_reset_gives_fresh_tables_and_outputs():
     w = inputs.TINY_BF16
     c = gca.Cache.for_workload(w)

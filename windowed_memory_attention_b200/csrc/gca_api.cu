@@ -41,7 +41,8 @@ using gca::WalkEntry;
 namespace {
 
 constexpr int kRing = 4;       // pinned staging slots for walk-list uploads
-constexpr int kQRing = 4;      // device staging slots for host query blocks
+constexpr int kQRing = 8;      // device staging slots for host query blocks
+constexpr int kORing = 2;      // device staging slots for host output blocks
 constexpr int kTileRows = 128;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -99,18 +100,27 @@ struct gca_cache {
     int* h_status = nullptr;
     int* d_status = nullptr;
     // staging for host-memory arguments: inputs are copied on the library's own
-    // copy stream (so uploads overlap the caller's compute stream), guarded by
-    // events; pinned host outputs are written by the kernels directly
+    // copy streams (so uploads overlap the kernels), guarded by events; outputs
+    // are written to device staging and copied back on copy_out
     cudaStream_t copy = nullptr;      // query-block uploads (ring of staging slots)
     cudaStream_t copy_kv = nullptr;   // K/V uploads, so they never queue behind the ring
+    cudaStream_t copy_out = nullptr;  // output blocks back to host memory
     void* st_k = nullptr;
     void* st_v = nullptr;
     cudaEvent_t kv_free = nullptr, kv_ready = nullptr;
     void* st_q[kQRing] = {};
     cudaEvent_t q_free[kQRing] = {}, q_ready[kQRing] = {};
     int q_pos = 0;
-    void* st_out = nullptr;
-    float* st_lse = nullptr;
+    void* st_out[kORing] = {};
+    float* st_lse[kORing] = {};
+    cudaEvent_t o_free[kORing] = {};
+    cudaEvent_t o_ready = nullptr;
+    int o_pos = 0;
+    // device work of calls whose pointer arguments all live in host memory
+    // (see begin_call); ev_fork / ev_join order it against the caller's stream
+    cudaStream_t xs = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    bool on_xs = false;               // the cache's latest device work is on xs
     long long launches = 0;
     bool host_only = false;   // GCA_HOST_ONLY: the page table alone, no device state
     // 3D rotary encoding: (cos, sin) tables of the time pairs per frame index
@@ -148,8 +158,16 @@ void release(gca_cache* c) {
         if (c->q_free[i]) cudaEventDestroy(c->q_free[i]);
         if (c->q_ready[i]) cudaEventDestroy(c->q_ready[i]);
     }
-    cudaFree(c->st_out);
-    cudaFree(c->st_lse);
+    for (int i = 0; i < kORing; ++i) {
+        cudaFree(c->st_out[i]);
+        cudaFree(c->st_lse[i]);
+        if (c->o_free[i]) cudaEventDestroy(c->o_free[i]);
+    }
+    if (c->o_ready) cudaEventDestroy(c->o_ready);
+    if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+    if (c->ev_join) cudaEventDestroy(c->ev_join);
+    if (c->copy_out) cudaStreamDestroy(c->copy_out);
+    if (c->xs) cudaStreamDestroy(c->xs);
     cudaFree(c->rope_t);
     cudaFree(c->rope_sp);
     if (c->kv_free) cudaEventDestroy(c->kv_free);
@@ -188,25 +206,52 @@ struct DeviceGuard {
     }
 };
 
-// Where a caller's pointer lives: device memory (used as is), pinned host
-// memory (the device reaches it through *alias), or pageable host memory.
+// Where a caller's pointer lives: device (or managed) memory is used in place;
+// pinned and pageable host memory are staged through library buffers.
 enum class Mem { kDevice, kPinned, kPageable };
 
-Mem classify(const void* ptr, void** alias = nullptr) {
+Mem classify(const void* ptr) {
     cudaPointerAttributes a{};
     if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
         cudaGetLastError();
         return Mem::kPageable;
     }
     if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return Mem::kDevice;
-    if (a.type == cudaMemoryTypeHost && a.devicePointer) {
-        if (alias) *alias = a.devicePointer;
-        return Mem::kPinned;
-    }
-    return Mem::kPageable;
+    return a.type == cudaMemoryTypeHost ? Mem::kPinned : Mem::kPageable;
 }
 
 bool is_device_ptr(const void* ptr) { return classify(ptr) == Mem::kDevice; }
+
+// The stream a call's device work runs on.  A call whose pointer arguments
+// all live in host memory reads nothing that earlier work on the caller's
+// stream writes: its inputs are staged and its outputs copied back by the
+// library.  Its work runs on the cache's own stream xs, after the cache's
+// earlier work only, so the copy back of one call overlaps the kernels of the
+// next; end_call makes the caller's stream wait for the call.  Any other call
+// runs on the caller's stream.
+bool begin_call(gca_cache* c, cudaStream_t st, bool detached, cudaStream_t* ex) {
+    *ex = st;
+    if (!detached) {
+        // the cache's work on xs, if any, is already waited for by st (end_call)
+        c->on_xs = false;
+        return true;
+    }
+    if (!c->on_xs && (cudaEventRecord(c->ev_fork, st) != cudaSuccess ||
+                      cudaStreamWaitEvent(c->xs, c->ev_fork, 0) != cudaSuccess))
+        return false;
+    c->on_xs = true;
+    *ex = c->xs;
+    return true;
+}
+
+int end_call(gca_cache* c, cudaStream_t st, cudaStream_t ex, int rc) {
+    if (ex != st && (cudaEventRecord(c->ev_join, ex) != cudaSuccess ||
+                     cudaStreamWaitEvent(st, c->ev_join, 0) != cudaSuccess))
+        return rc ? rc : GCA_ERR_CUDA;
+    return rc;
+}
+
+bool on_host(const void* ptr) { return ptr && classify(ptr) != Mem::kDevice; }
 
 // Upload a host query block into a staging slot on the cache's copy stream: the
 // copy waits until the buffer's previous reader (on the caller's stream) is
@@ -336,7 +381,8 @@ int upload_walk(gca_cache* c, const std::vector<gca_page_entry_t>& w, WalkEntry*
 // Attention of F query frames (the first is first_query_frame) over a device
 // walk list; stages host q / out / lse through the cache's buffers.
 int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query_frame,
-                  const WalkEntry* walk, int nwalk, void* out, float* lse, cudaStream_t st) {
+                  const WalkEntry* walk, int nwalk, void* out, float* lse, cudaStream_t ex,
+                  cudaStream_t st) {
     const gca_config_t& g = c->cfg;
     const int R = F * c->Lq;
     const size_t qbytes = (size_t)R * g.num_heads * gca::kHeadDim * c->elem;
@@ -345,27 +391,30 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     if (!is_device_ptr(q)) {
         qslot = c->q_pos;
         c->q_pos = (c->q_pos + 1) % kQRing;
-        if (!stage_in(c, c->st_q[qslot], q, qbytes, c->q_free[qslot], c->q_ready[qslot], st))
+        if (!stage_in(c, c->st_q[qslot], q, qbytes, c->q_free[qslot], c->q_ready[qslot], ex))
             return GCA_ERR_CUDA;
         qd = c->st_q[qslot];
     }
-    // outputs: device memory and pinned host memory (through its device alias)
-    // are written by the kernels; pageable host memory is staged and copied back
-    void* out_alias = nullptr;
-    void* lse_alias = nullptr;
-    const Mem out_mem = classify(out, &out_alias);
-    const Mem lse_mem = lse ? classify(lse, &lse_alias) : Mem::kDevice;
-    const bool out_host = out_mem == Mem::kPageable;
-    const bool lse_host = lse && lse_mem == Mem::kPageable;
-    void* out_k = out_mem == Mem::kPinned ? out_alias : out;
-    float* lse_k = lse_mem == Mem::kPinned ? static_cast<float*>(lse_alias) : lse;
+    // outputs in host memory (pinned or pageable) are written to a device
+    // staging slot by the kernel and copied back by the copy engine, which
+    // moves them at PCIe rate; kernel stores into a mapped pinned buffer
+    // stall the CTAs that issue them
+    const bool out_host = on_host(out);
+    const bool lse_host = on_host(lse);
+    int oslot = -1;
+    if (out_host || lse_host) {
+        oslot = c->o_pos;
+        c->o_pos = (c->o_pos + 1) % kORing;
+        // the slot's previous copy back has read it
+        if (cudaStreamWaitEvent(ex, c->o_free[oslot], 0) != cudaSuccess) return GCA_ERR_CUDA;
+    }
 
     gca::AttendParams p{};
     p.walk = walk;
     p.nwalk = nwalk;
     p.q = qd;
-    p.out = out_host ? c->st_out : out_k;
-    p.lse = lse ? (lse_host ? c->st_lse : lse_k) : nullptr;
+    p.out = out_host ? c->st_out[oslot] : out;
+    p.lse = lse ? (lse_host ? c->st_lse[oslot] : lse) : nullptr;
     p.R = R;
     p.H = g.num_heads;
     p.Lq = c->Lq;
@@ -393,25 +442,35 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
         p.W = ceil_div(total, p.seg);
         p.merge_cnt = c->merge_cnt;
         p.epoch = ++c->epoch;
-        err = gca::launch_attend_sm100(c->tmK, c->tmV, p, st);
+        err = gca::launch_attend_sm100(c->tmK, c->tmV, p, ex);
         c->launches += 1;
     } else {
         p.QT = ceil_div(R, kTileRows);
         p.W = 1;
         p.seg = 1;
-        err = gca::launch_attend_f32(p, c->kpool, c->vpool, st);
+        err = gca::launch_attend_f32(p, c->kpool, c->vpool, ex);
         c->launches += 1;
     }
     if (err != cudaSuccess) {
         cudaGetLastError();
         return GCA_ERR_CUDA;
     }
-    if (qslot >= 0 && cudaEventRecord(c->q_free[qslot], st) != cudaSuccess) return GCA_ERR_CUDA;
-    if (out_host && cudaMemcpyAsync(out, c->st_out, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return GCA_ERR_CUDA;
-    if (lse_host && cudaMemcpyAsync(lse, c->st_lse, (size_t)R * g.num_heads * sizeof(float),
-                                    cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return GCA_ERR_CUDA;
+    if (qslot >= 0 && cudaEventRecord(c->q_free[qslot], ex) != cudaSuccess) return GCA_ERR_CUDA;
+    if (oslot >= 0) {
+        // copy back on copy_out when the call runs on xs (the next call's
+        // kernels go on while it runs), else in the caller's stream order
+        cudaStream_t cs = ex == st ? st : c->copy_out;
+        if (cs != ex && (cudaEventRecord(c->o_ready, ex) != cudaSuccess ||
+                         cudaStreamWaitEvent(cs, c->o_ready, 0) != cudaSuccess))
+            return GCA_ERR_CUDA;
+        if (out_host && cudaMemcpyAsync(out, c->st_out[oslot], qbytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+            return GCA_ERR_CUDA;
+        if (lse_host && cudaMemcpyAsync(lse, c->st_lse[oslot], (size_t)R * g.num_heads * sizeof(float),
+                                        cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+            return GCA_ERR_CUDA;
+        if (cudaEventRecord(c->o_free[oslot], cs) != cudaSuccess) return GCA_ERR_CUDA;
+        if (cs != st && cudaStreamWaitEvent(st, c->o_free[oslot], 0) != cudaSuccess) return GCA_ERR_CUDA;
+    }
     return GCA_OK;
 }
 
@@ -569,9 +628,17 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
              cudaEventCreateWithFlags(&c->q_free[i], cudaEventDisableTiming) == cudaSuccess &&
              cudaEventCreateWithFlags(&c->q_ready[i], cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaMalloc(&c->st_k, frame_bytes * g.num_layers) == cudaSuccess &&
-         cudaMalloc(&c->st_v, frame_bytes * g.num_layers) == cudaSuccess &&
-         cudaMalloc(&c->st_out, frame_bytes * g.max_query_frames) == cudaSuccess &&
-         cudaMalloc((void**)&c->st_lse, (size_t)c->Lq * g.num_heads * g.max_query_frames * sizeof(float)) == cudaSuccess;
+         cudaMalloc(&c->st_v, frame_bytes * g.num_layers) == cudaSuccess;
+    for (int i = 0; ok && i < kORing; ++i)
+        ok = cudaMalloc(&c->st_out[i], frame_bytes * g.max_query_frames) == cudaSuccess &&
+             cudaMalloc((void**)&c->st_lse[i], (size_t)c->Lq * g.num_heads * g.max_query_frames * sizeof(float)) ==
+                 cudaSuccess &&
+             cudaEventCreateWithFlags(&c->o_free[i], cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaStreamCreateWithFlags(&c->copy_out, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&c->xs, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->o_ready, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) == cudaSuccess;
     if (!ok) {
         cudaGetLastError();
         release(c);
@@ -651,9 +718,11 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
         return GCA_OK;
     }
 
+    cudaStream_t ex;
+    if (!begin_call(c, st, on_host(k) && on_host(v), &ex)) return GCA_ERR_CUDA;
     gca::AppendParams p{};
     const size_t bytes = (size_t)nl * c->Lq * g.num_heads * gca::kHeadDim * c->elem;
-    if (!stage_kv(c, k, v, bytes, st, &p.k, &p.v)) return GCA_ERR_CUDA;
+    if (!stage_kv(c, k, v, bytes, ex, &p.k, &p.v)) return end_call(c, st, ex, GCA_ERR_CUDA);
     p.kpool = c->kpool;
     p.vpool = c->vpool;
     p.layer0 = l0;
@@ -678,15 +747,15 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
     for (int i = 0; i < c->ipf; ++i) p.img_pages[i] = img[i];
     p.rope = c->rope();
     p.rope_t = t;
-    if (gca::launch_append(p, st) != cudaSuccess) {
+    if (gca::launch_append(p, ex) != cudaSuccess) {
         cudaGetLastError();
-        return GCA_ERR_CUDA;
+        return end_call(c, st, ex, GCA_ERR_CUDA);
     }
     c->launches += 1;
-    if (cudaEventRecord(c->kv_free, st) != cudaSuccess) return GCA_ERR_CUDA;
+    if (cudaEventRecord(c->kv_free, ex) != cudaSuccess) return end_call(c, st, ex, GCA_ERR_CUDA);
     for (int l = l0; l < l0 + nl; ++l) c->layer_frames[l] = t + 1;
     if (frame_index_out) *frame_index_out = t;
-    return GCA_OK;
+    return end_call(c, st, ex, GCA_OK);
 }
 
 int gca_evict_to_summary(gca_cache_t* c, int32_t* frames_evicted_out) {
@@ -810,16 +879,18 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
     DeviceGuard guard(c->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
+    cudaStream_t ex;
+    if (!begin_call(c, st, on_host(q) && on_host(out) && (!lse || on_host(lse)), &ex)) return GCA_ERR_CUDA;
     // walk list: rebuilt and uploaded when the page table or the block changed
     if (c->up_version != c->version || c->up_F != F) {
         std::vector<gca_page_entry_t> w;
-        if (!build_walk(c, F, w)) return GCA_ERR_STATE;
-        if (int e = upload_walk(c, w, c->d_walk, st)) return e;
+        if (!build_walk(c, F, w)) return end_call(c, st, ex, GCA_ERR_STATE);
+        if (int e = upload_walk(c, w, c->d_walk, ex)) return end_call(c, st, ex, e);
         c->up_version = c->version;
         c->up_F = F;
         c->up_n = (int)w.size();
     }
-    return run_attention(c, layer, q, F, c->T - F, c->d_walk, c->up_n, out, lse, st);
+    return end_call(c, st, ex, run_attention(c, layer, q, F, c->T - F, c->d_walk, c->up_n, out, lse, ex, st));
 }
 
 int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
@@ -831,8 +902,11 @@ int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void
     if (int s = check_status(c)) return s;
     DeviceGuard guard(c->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (int e = stage_transient(c, layer, k, v, 0, st)) return e;
-    return run_attention(c, layer, q, 1, 0, c->d_walk_f, c->tpf, out, lse, st);
+    cudaStream_t ex;
+    if (!begin_call(c, st, on_host(q) && on_host(k) && on_host(v) && on_host(out) && (!lse || on_host(lse)), &ex))
+        return GCA_ERR_CUDA;
+    if (int e = stage_transient(c, layer, k, v, 0, ex)) return end_call(c, st, ex, e);
+    return end_call(c, st, ex, run_attention(c, layer, q, 1, 0, c->d_walk_f, c->tpf, out, lse, ex, st));
 }
 
 int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
@@ -852,19 +926,22 @@ int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const voi
     // which the walk list carries as full-frame pages of frame t.  With no
     // keyframe yet it reads only itself.
     const int i = c->T > 0 ? c->T - 1 : 0;
+    cudaStream_t ex;
+    if (!begin_call(c, st, on_host(q) && on_host(k) && on_host(v) && on_host(out) && (!lse || on_host(lse)), &ex))
+        return GCA_ERR_CUDA;
     if (c->tup_version != c->version) {
         std::vector<gca_page_entry_t> w;
-        if (c->T > 0 && !build_walk(c, 1, w)) return GCA_ERR_STATE;
+        if (c->T > 0 && !build_walk(c, 1, w)) return end_call(c, st, ex, GCA_ERR_STATE);
         for (int s = 0; s < c->tpf; ++s) {
             const int first = s * c->P;
             w.push_back({c->num_regular + s, GCA_PAGE_IMAGE, i, first, std::min(c->P, c->Lq - first)});
         }
-        if (int e = upload_walk(c, w, c->d_walk_t, st)) return e;
+        if (int e = upload_walk(c, w, c->d_walk_t, ex)) return end_call(c, st, ex, e);
         c->tup_version = c->version;
         c->tup_n = (int)w.size();
     }
 
-    if (int e = stage_transient(c, layer, k, v, i, st)) return e;
-    return run_attention(c, layer, q, 1, i, c->d_walk_t, c->tup_n, out, lse, st);
+    if (int e = stage_transient(c, layer, k, v, i, ex)) return end_call(c, st, ex, e);
+    return end_call(c, st, ex, run_attention(c, layer, q, 1, i, c->d_walk_t, c->tup_n, out, lse, ex, st));
 }
 }  // extern "C"
