@@ -107,7 +107,7 @@ def lk_at(w, T):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -121,7 +121,7 @@ class ClockSampler:
             sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -425,6 +425,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": tr["dram_bytes_per_launch"] if tr else None,
                      "kernel": "gca attend (tcgen05, split heads merged in the kernel), per layer launch",
                      "peak_source": f"{pk['source']} bf16 burst; sustained {pk['bf16_sustained']}",
+                     "frac_of_sustained": att_tflops / pk["bf16_sustained"] if pk["bf16_sustained"] else None,
                      "algorithmic_flop_per_launch": flops / (K * w.L),
                      "avg_launch_ms": statistics.mean(att_ms)},
         "append_roofline": {"bound": "hbm", "achieved": app_gbs, "peak": pk["hbm"],
