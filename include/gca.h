@@ -24,7 +24,9 @@
  * to library device buffers and copied back the same way.  The stream argument
  * waits for those copies, so the caller synchronises the stream before
  * reading a host output.  Device pointers must stay valid until the stream has
- * consumed them.
+ * consumed them, and start on a 16-byte boundary (lse: 4-byte), as every
+ * allocation does: the kernels move 16-byte vectors, and a device pointer off
+ * that boundary is refused with GCA_ERR_INVALID_ARG before anything runs.
  *
  * A call whose pointer arguments are ALL in host memory does not wait for
  * earlier work on the stream: its kernels follow the cache's earlier calls

@@ -413,6 +413,55 @@ def test_transient_before_any_keyframe_and_host_pointers(w):
     assert cache.info().frames == 0
 
 
+def _misaligned(x: torch.Tensor) -> torch.Tensor:
+    """The same values at an address 8 bytes past a 16-byte boundary."""
+    flat = torch.empty(x.numel() + 4, dtype=x.dtype, device=x.device)
+    view = flat[4:].view(x.shape)
+    view.copy_(x)
+    assert view.data_ptr() % 16 == 8
+    return view
+
+
+@pytest.mark.parametrize("w", [inputs.TINY_BF16, inputs.METRIC_518x378.with_(L=1)], ids=["bf16", "518x378"])
+def test_frame_tokens_read_in_place_and_misaligned_tensors_refused(w):
+    """bf16 K/V of the query frame are read in place by the attention kernel
+    (a 3D tensor map over [S+M][H][D]): one launch per non-keyframe or
+    intra-frame call (their values against the oracle: the transient and
+    intra-frame tests).  A device tensor off a 16-byte boundary is refused
+    before anything is launched or changed."""
+    cache = gca.Cache.for_workload(w)
+    for t in range(w.n + 2):
+        cache.append(inputs.draw(w, t, "k").cuda(), inputs.draw(w, t, "v").cuda())
+        cache.evict()
+    q, k, v = (inputs.draw(w, w.n + 7, x)[0].cuda() for x in "qkv")
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    for call in (cache.attend_transient, cache.frame_attention):
+        n0 = cache.info().kernel_launches
+        call(0, q, k, v, out, lse)
+        assert cache.info().kernel_launches - n0 == 1
+    torch.cuda.synchronize()
+    layout, n0 = cache.layout(), cache.info().kernel_launches
+    bad = [(_misaligned(q), k, v), (q, _misaligned(k), v), (q, k, _misaligned(v))]
+    for qq, kk, vv in bad:
+        for call in (cache.attend_transient, cache.frame_attention):
+            with pytest.raises(gca.GCAError) as e:
+                call(0, qq, kk, vv, out, lse)
+            assert e.value.name == "GCA_ERR_INVALID_ARG"
+    kw, vw = inputs.draw(w, w.n + 2, "k").cuda(), inputs.draw(w, w.n + 2, "v").cuda()
+    for refused in (lambda: cache.attend(0, _misaligned(q)[None], out[None]),
+                    lambda: cache.attend(0, q[None], _misaligned(out)[None]),
+                    lambda: cache.append(_misaligned(kw), vw),
+                    lambda: cache.append(kw, _misaligned(vw))):
+        with pytest.raises(gca.GCAError) as e:
+            refused()
+        assert e.value.name == "GCA_ERR_INVALID_ARG"
+    assert cache.info().kernel_launches == n0 and cache.layout() == layout
+    assert cache.info().frames == w.n + 2
+    cache.append(kw, vw)                    # the cache goes on as before
+    assert cache.status() == 0
+
+
 # ----------------------------------------------------------------------------
 # intra-frame attention (the layers that alternate with GCA)
 # ----------------------------------------------------------------------------

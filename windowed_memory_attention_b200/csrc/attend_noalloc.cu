@@ -136,6 +136,12 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     if (!is_device_ptr(k_pool) || !is_device_ptr(v_pool) || !is_device_ptr(q) || !is_device_ptr(out) ||
         (lse && !is_device_ptr(lse)) || (status && !is_device_ptr(status)))
         return GCA_ERR_INVALID_ARG;
+    // the kernel moves 16-byte vectors through the pools (TMA), q and out,
+    // and 4-byte words through lse, status and a device walk list
+    auto off = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (off(k_pool, 16) || off(v_pool, 16) || off(q, 16) || off(out, 16) || off(lse, 4) || off(status, 4) ||
+        off(walk, 4))
+        return GCA_ERR_INVALID_ARG;
     if (nwalk > kNoallocMaxWalk) return GCA_ERR_CAPACITY;
     const long long R = (long long)num_query_frames * tokens_per_frame;
     const int QT = (int)((R + 127) / 128);
@@ -229,7 +235,8 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     p.W = (int)((total + p.seg - 1) / p.seg);
     p.merge_cnt = counts;
     p.epoch = g_epoch.fetch_add(1) + 1;
-    cudaError_t err = gca::launch_attend_sm100(tk, tv, p, st);
+    p.frame_page0 = INT_MAX;
+    cudaError_t err = gca::launch_attend_sm100(tk, tv, tk, tv, p, st);
     if (err != cudaSuccess) {
         cudaGetLastError();
         return GCA_ERR_CUDA;

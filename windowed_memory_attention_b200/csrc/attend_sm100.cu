@@ -167,6 +167,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm,
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y, int z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format:
 // start >> 4 in [0,14), leading byte offset >> 4 in [16,30), stride byte
 // offset >> 4 in [32,46), version 1 at [46,48), swizzle mode 2 at [61,64)).
@@ -305,6 +314,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 template <int PAGE>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+              const __grid_constant__ CUtensorMap tmKf, const __grid_constant__ CUtensorMap tmVf,
               const AttendParams p) {
     using L = Layout<PAGE>;
     extern __shared__ uint8_t smem_raw[];
@@ -385,6 +395,10 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     if (warp == kWarpTMA && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+        if (p.frame_page0 < p.num_pages) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmKf)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmVf)) : "memory");
+        }
     }
     fence_before();
     __syncthreads();
@@ -404,18 +418,26 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     ok = false;
                     break;
                 }
-                const int page = __ldg(&p.walk[e].x);
+                const int4 ent = __ldg(&p.walk[e]);
+                const int page = ent.x;
                 if (page < 0 || page >= p.num_pages) {
                     *abort_flag = 1;
                     *(volatile int*)p.status = kStatusBadPage;
                     ok = false;
                     break;
                 }
-                const int y = ((p.layer * p.num_pages + page) * p.H + h) * PAGE;
                 const uint32_t dst = sbase + st * L::kStageBytes;
                 mbar_expect_tx(kv_full(st), 2 * L::kTileBytes);
-                tma_load_2d(dst, &tmK, 0, y, kv_full(st));
-                tma_load_2d(dst + L::kTileBytes, &tmV, 0, y, kv_full(st));
+                if (page >= p.frame_page0) {
+                    // the frame's own tokens first .. first+PAGE-1 of head h
+                    // (past the last token the box reads zeros)
+                    tma_load_3d(dst, &tmKf, 0, h, ent.z, kv_full(st));
+                    tma_load_3d(dst + L::kTileBytes, &tmVf, 0, h, ent.z, kv_full(st));
+                } else {
+                    const int y = ((p.layer * p.num_pages + page) * p.H + h) * PAGE;
+                    tma_load_2d(dst, &tmK, 0, y, kv_full(st));
+                    tma_load_2d(dst + L::kTileBytes, &tmV, 0, y, kv_full(st));
+                }
                 ++issued;
                 if (++e == p.nwalk) {
                     e = 0;
@@ -821,23 +843,23 @@ __global__ void bounded_wait_selftest(int* status, unsigned long long timeout_ns
 }
 
 template <int PAGE>
-cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const AttendParams& p,
-                        cudaStream_t s) {
+cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkf,
+                        const CUtensorMap& tvf, const AttendParams& p, cudaStream_t s) {
     const int smem = Layout<PAGE>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(attend_kernel<PAGE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((p.QT + 1) / 2, p.W);
-    attend_kernel<PAGE><<<grid, kThreads, smem, s>>>(tk, tv, p);
+    attend_kernel<PAGE><<<grid, kThreads, smem, s>>>(tk, tv, tkf, tvf, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
-                                const AttendParams& p, cudaStream_t s) {
-    if (p.P == 128) return launch_page<128>(tk, tv, p, s);
-    if (p.P == 64) return launch_page<64>(tk, tv, p, s);
+cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkf,
+                                const CUtensorMap& tvf, const AttendParams& p, cudaStream_t s) {
+    if (p.P == 128) return launch_page<128>(tk, tv, tkf, tvf, p, s);
+    if (p.P == 64) return launch_page<64>(tk, tv, tkf, tvf, p, s);
     return cudaErrorInvalidValue;
 }
 

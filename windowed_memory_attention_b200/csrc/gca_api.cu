@@ -80,6 +80,7 @@ struct gca_cache {
     void* vpool = nullptr;
     size_t pool_bytes = 0;
     CUtensorMap tmK{}, tmV{};
+    EncodeTiledFn encode = nullptr;   // cuTensorMapEncodeTiled (driver entry point)
     WalkEntry* d_walk = nullptr;
     int walk_cap = 0;
     WalkEntry* h_stage[kRing] = {};
@@ -253,6 +254,14 @@ int end_call(gca_cache* c, cudaStream_t st, cudaStream_t ex, int rc) {
 
 bool on_host(const void* ptr) { return ptr && classify(ptr) != Mem::kDevice; }
 
+// The kernels move 16-byte vectors through q, k, v and out and 4-byte words
+// through lse: a device pointer must start on such a boundary (allocations
+// do).  Host pointers may sit anywhere: they are staged through aligned
+// library buffers.
+bool placed(const void* ptr, uintptr_t align) {
+    return !ptr || (reinterpret_cast<uintptr_t>(ptr) % align) == 0 || on_host(ptr);
+}
+
 // Upload a host query block into a staging slot on the cache's copy stream: the
 // copy waits until the buffer's previous reader (on the caller's stream) is
 // done (`free_ev`), and the caller's stream waits for the copy (`ready_ev`).
@@ -295,6 +304,22 @@ bool encode_pool_map(EncodeTiledFn enc, CUtensorMap* tm, void* pool, const gca_c
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
+}
+
+// A frame's K or V as the caller passes it, [S+M][H][D] bf16, viewed as a 3D
+// tensor (D, H, token): a box of D x 1 x P is one head's tile of P tokens,
+// laid out in shared memory exactly like a pool page tile; boxes past the
+// last token read zeros.
+bool encode_frame_map(const gca_cache* c, CUtensorMap* tm, const void* base) {
+    if (!c->encode || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
+    const cuuint64_t H = (cuuint64_t)c->cfg.num_heads;
+    cuuint64_t dims[3] = {(cuuint64_t)gca::kHeadDim, H, (cuuint64_t)c->Lq};
+    cuuint64_t strides[2] = {(cuuint64_t)gca::kHeadDim * 2, H * gca::kHeadDim * 2};
+    cuuint32_t box[3] = {(cuuint32_t)gca::kHeadDim, 1, (cuuint32_t)c->P};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return c->encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Host tables of the 3D rotary encoding.  Axis a (time, patch row, patch
@@ -380,9 +405,11 @@ int upload_walk(gca_cache* c, const std::vector<gca_page_entry_t>& w, WalkEntry*
 
 // Attention of F query frames (the first is first_query_frame) over a device
 // walk list; stages host q / out / lse through the cache's buffers.
+// fk / fv (nullable): the query frame's own K and V, read in place by the
+// kernel for the transient pages (ids >= num_regular) of the walk list.
 int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query_frame,
                   const WalkEntry* walk, int nwalk, void* out, float* lse, cudaStream_t ex,
-                  cudaStream_t st) {
+                  cudaStream_t st, const CUtensorMap* fk = nullptr, const CUtensorMap* fv = nullptr) {
     const gca_config_t& g = c->cfg;
     const int R = F * c->Lq;
     const size_t qbytes = (size_t)R * g.num_heads * gca::kHeadDim * c->elem;
@@ -442,7 +469,8 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
         p.W = ceil_div(total, p.seg);
         p.merge_cnt = c->merge_cnt;
         p.epoch = ++c->epoch;
-        err = gca::launch_attend_sm100(c->tmK, c->tmV, p, ex);
+        p.frame_page0 = fk && fv ? c->num_regular : INT_MAX;
+        err = gca::launch_attend_sm100(c->tmK, c->tmV, fk ? *fk : c->tmK, fv ? *fv : c->tmV, p, ex);
         c->launches += 1;
     } else {
         p.QT = ceil_div(R, kTileRows);
@@ -474,13 +502,21 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     return GCA_OK;
 }
 
-// A frame's K and V into this layer's transient pages: token u of the frame
-// (summary tokens first) at page u / P, slot u % P.
-int stage_transient(gca_cache* c, int layer, const void* k, const void* v, int frame, cudaStream_t st) {
+// A frame's K and V for attention over its own tokens.  bf16 without RoPE:
+// the attention kernel reads them in place through *fk / *fv (host inputs
+// are staged first) and *direct is set; the caller records kv_free after the
+// attention kernel.  Otherwise append_kernel writes them into this layer's
+// transient pages: token u of the frame (summary tokens first) at page u / P,
+// slot u % P.
+int stage_transient(gca_cache* c, int layer, const void* k, const void* v, int frame, cudaStream_t st,
+                    CUtensorMap* fk, CUtensorMap* fv, bool* direct) {
     const gca_config_t& g = c->cfg;
     gca::AppendParams p{};
     const size_t bytes = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
     if (!stage_kv(c, k, v, bytes, st, &p.k, &p.v)) return GCA_ERR_CUDA;
+    *direct = g.dtype == GCA_DTYPE_BF16 && g.rope == GCA_ROPE_NONE && encode_frame_map(c, fk, p.k) &&
+              encode_frame_map(c, fv, p.v);
+    if (*direct) return GCA_OK;
     p.kpool = c->kpool;
     p.vpool = c->vpool;
     p.layer0 = layer;
@@ -659,6 +695,7 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
             release(c);
             return GCA_ERR_CUDA;
         }
+        c->encode = (EncodeTiledFn)fn;
     }
     *out = c;
     return GCA_OK;
@@ -673,6 +710,7 @@ int gca_append_frame(gca_cache_t* c, int32_t layer, const void* k, const void* v
                      int64_t* frame_index_out, void* stream) {
     Range range("gca_append_frame");
     if (!c || (!c->host_only && (!k || !v))) return GCA_ERR_INVALID_ARG;
+    if (!c->host_only && (!placed(k, 16) || !placed(v, 16))) return GCA_ERR_INVALID_ARG;
     const gca_config_t& g = c->cfg;
     if (layer != GCA_ALL_LAYERS && (layer < 0 || layer >= g.num_layers)) return GCA_ERR_INVALID_ARG;
     if (int s = check_status(c)) return s;
@@ -870,6 +908,7 @@ int gca_attend(gca_cache_t* c, int32_t layer, const void* q, int32_t F, void* ou
                void* stream) {
     Range range("gca_attend");
     if (!c || !q || !out) return GCA_ERR_INVALID_ARG;
+    if (!placed(q, 16) || !placed(out, 16) || !placed(lse, 4)) return GCA_ERR_INVALID_ARG;
     if (c->host_only) return GCA_ERR_UNSUPPORTED;
     const gca_config_t& g = c->cfg;
     if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
@@ -897,6 +936,8 @@ int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void
                         void* out, float* lse, void* stream) {
     Range range("gca_frame_attention");
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
+    if (!placed(q, 16) || !placed(k, 16) || !placed(v, 16) || !placed(out, 16) || !placed(lse, 4))
+        return GCA_ERR_INVALID_ARG;
     if (c->host_only) return GCA_ERR_UNSUPPORTED;
     if (layer < 0 || layer >= c->cfg.num_layers) return GCA_ERR_INVALID_ARG;
     if (int s = check_status(c)) return s;
@@ -905,14 +946,21 @@ int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void
     cudaStream_t ex;
     if (!begin_call(c, st, on_host(q) && on_host(k) && on_host(v) && on_host(out) && (!lse || on_host(lse)), &ex))
         return GCA_ERR_CUDA;
-    if (int e = stage_transient(c, layer, k, v, 0, ex)) return end_call(c, st, ex, e);
-    return end_call(c, st, ex, run_attention(c, layer, q, 1, 0, c->d_walk_f, c->tpf, out, lse, ex, st));
+    CUtensorMap fk{}, fv{};
+    bool direct = false;
+    if (int e = stage_transient(c, layer, k, v, 0, ex, &fk, &fv, &direct)) return end_call(c, st, ex, e);
+    int rc = run_attention(c, layer, q, 1, 0, c->d_walk_f, c->tpf, out, lse, ex, st, direct ? &fk : nullptr,
+                           direct ? &fv : nullptr);
+    if (direct && rc == GCA_OK && cudaEventRecord(c->kv_free, ex) != cudaSuccess) rc = GCA_ERR_CUDA;
+    return end_call(c, st, ex, rc);
 }
 
 int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,
                          void* out, float* lse, void* stream) {
     Range range("gca_attend_transient");
     if (!c || !q || !k || !v || !out) return GCA_ERR_INVALID_ARG;
+    if (!placed(q, 16) || !placed(k, 16) || !placed(v, 16) || !placed(out, 16) || !placed(lse, 4))
+        return GCA_ERR_INVALID_ARG;
     if (c->host_only) return GCA_ERR_UNSUPPORTED;
     const gca_config_t& g = c->cfg;
     if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
@@ -941,7 +989,12 @@ int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const voi
         c->tup_n = (int)w.size();
     }
 
-    if (int e = stage_transient(c, layer, k, v, i, ex)) return end_call(c, st, ex, e);
-    return end_call(c, st, ex, run_attention(c, layer, q, 1, i, c->d_walk_t, c->tup_n, out, lse, ex, st));
+    CUtensorMap fk{}, fv{};
+    bool direct = false;
+    if (int e = stage_transient(c, layer, k, v, i, ex, &fk, &fv, &direct)) return end_call(c, st, ex, e);
+    int rc = run_attention(c, layer, q, 1, i, c->d_walk_t, c->tup_n, out, lse, ex, st, direct ? &fk : nullptr,
+                           direct ? &fv : nullptr);
+    if (direct && rc == GCA_OK && cudaEventRecord(c->kv_free, ex) != cudaSuccess) rc = GCA_ERR_CUDA;
+    return end_call(c, st, ex, rc);
 }
 }  // extern "C"

@@ -1,6 +1,7 @@
 // Internal declarations shared by the host code and the kernels of libgca.
 #pragma once
 
+#include <climits>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -106,12 +107,20 @@ struct AttendParams {
     // with the launch's epoch in the high word (no reset between launches)
     unsigned long long* merge_cnt;   // [QT][H]
     unsigned int epoch;
+    // walk-list pages with id >= frame_page0 hold the query frame's own
+    // tokens: they are read from the caller's [S+M][H][D] K and V through the
+    // frame tensor maps (token `first` of the walk entry onwards) instead of
+    // the pools.  INT_MAX when unused.
+    int frame_page0;
 };
 
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
-cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv,
-                                const AttendParams& p, cudaStream_t s);
+// tk / tv: the pools as [L * num_pages * H * P][D]; tkf / tvf: a frame's
+// [S+M][H][D] K and V (read for pages >= p.frame_page0; any valid map when
+// p.frame_page0 is INT_MAX)
+cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkf,
+                                const CUtensorMap& tvf, const AttendParams& p, cudaStream_t s);
 cudaError_t launch_bounded_wait_selftest(int* status, unsigned long long timeout_ns, cudaStream_t s);
 cudaError_t launch_attend_f32(const AttendParams& p, const void* kpool, const void* vpool,
                               cudaStream_t s);
