@@ -614,6 +614,8 @@ def run_report(args):
         cache.close()
 
     stream(inputs.WORKED_EXAMPLE, {100, 1000, 10000}, 10000)
+    # the 518x378 workload's layer at the same points (the bench line is its 24-layer T=10000 step)
+    stream(inputs.METRIC_518x378.with_(L=1), {100, 1000, 10000}, 10000)
     stream(inputs.DENSE_CAUSAL, {1000}, 1000)
     run_vo_stream(dev)
 
