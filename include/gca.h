@@ -227,10 +227,12 @@ int gca_attend(gca_cache_t* cache, int32_t layer, const void* q, int32_t num_que
  * reads only its own tokens.
  * q, k, v: [S+M][H][D] of this layer (summary tokens first), device or host
  * memory; out [S+M][H][D] in the cache dtype; lse (nullable) [S+M][H]
- * float32, natural log.  k and v are copied into ceil((S+M)/P) transient pages
- * of this layer (past the allocator's pages) and are dropped by the next call
- * for the layer: the page table, frame count and eviction state do not
- * change, so calls for one layer must be ordered (one stream).
+ * float32, natural log.  For a bf16 cache without RoPE the attention kernel
+ * reads k and v where they are (one launch; host tensors are staged first);
+ * otherwise they are copied into ceil((S+M)/P) transient pages of this layer
+ * (past the allocator's pages), which the next call for the layer reuses.
+ * The page table, frame count and eviction state do not change, so calls for
+ * one layer must be ordered (one stream).
  * Errors: STATE (layer has not appended frame T-1, or a frame the latest
  * keyframe needs was evicted), INVALID_ARG, DEVICE_CHECK. */
 int gca_attend_transient(gca_cache_t* cache, int32_t layer, const void* q, const void* k,
@@ -242,8 +244,8 @@ int gca_attend_transient(gca_cache_t* cache, int32_t layer, const void* q, const
  * token of the same frame, bidirectionally, softmax(scale * q.k), fp32
  * accumulation; no other frame is read.  q, k, v, out: [S+M][H][D] in the
  * cache dtype, device or host memory; lse (nullable) [S+M][H] float32.  k and
- * v go through the layer's transient pages like gca_attend_transient (and
- * overwrite what a transient call left there); the cache's page table and
+ * v are read like gca_attend_transient's (in place for a bf16 cache without
+ * RoPE, else through the layer's transient pages); the cache's page table and
  * frames are neither read nor changed.  Errors: INVALID_ARG, DEVICE_CHECK. */
 int gca_frame_attention(gca_cache_t* cache, int32_t layer, const void* q, const void* k,
                         const void* v, void* out, float* lse, void* stream);
