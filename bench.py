@@ -593,6 +593,14 @@ def run_report(args):
                       "note": "one launch: the frame's K/V read in place by the attention kernel "
                               "(bf16, no RoPE); 4.1 GFLOP per layer"}),
           flush=True)
+    # the same layer over 16 frames in one call (one launch: a CTA per frame, tile pair and head)
+    Fb = 16
+    qb, kb, vb = (torch.stack([inputs.draw(w, 3 + f, x, dev)[0] for f in range(Fb)]) for x in "qkv")
+    outb = torch.empty_like(qb)
+    att_b = _time_ms(lambda: cache.frame_attention_batch(0, qb, kb, vb, outb))
+    print(json.dumps({"workload": w.name + f" ({Fb} frames, one call)", "step": "intra-frame attention, batched",
+                      "frames": Fb, "ms_per_call": att_b, "ms_per_frame": att_b / Fb,
+                      "tflops": Fb * fl / att_b / 1e9}), flush=True)
     cache.close()
 
     # trajectory-memory variants on the 518x378 workload (one layer) at T=10000

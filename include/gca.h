@@ -250,6 +250,18 @@ int gca_attend_transient(gca_cache_t* cache, int32_t layer, const void* q, const
 int gca_frame_attention(gca_cache_t* cache, int32_t layer, const void* q, const void* k,
                         const void* v, void* out, float* lse, void* stream);
 
+/* Intra-frame attention of num_frames frames for one layer, each frame
+ * attending only to its own tokens, as gca_frame_attention does for one.
+ * q, k, v, out: [F][S+M][H][D] (F = num_frames >= 1) in the cache dtype;
+ * lse (nullable) [F][S+M][H] float32.  For a bf16 cache without RoPE and
+ * device tensors, up to 64 frames go in one launch with one CTA per (frame,
+ * query-tile pair, head), k and v read in place; otherwise (host tensors, an
+ * fp32 cache, RoPE) each frame is one gca_frame_attention call.  The cache's
+ * page table and frames are neither read nor changed.
+ * Errors: INVALID_ARG, DEVICE_CHECK, CUDA. */
+int gca_frame_attention_batch(gca_cache_t* cache, int32_t layer, int32_t num_frames, const void* q,
+                              const void* k, const void* v, void* out, float* lse, void* stream);
+
 /* Back to the creation state (windowed mode: state is reset at each window
  * start; code walkthrough §3.3).  Page tables become identical to a fresh
  * cache's; pool bytes are left as they are and never read before rewritten. */

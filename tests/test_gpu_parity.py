@@ -493,6 +493,44 @@ def test_frame_attention_is_dense_attention_within_the_frame(w):
     assert cache.layout() == sim.walk() and cache.info().frames == 3 and cache.status() == 0
 
 
+@pytest.mark.parametrize("w", [inputs.TINY, inputs.TINY_BF16, inputs.METRIC_518x378.with_(L=1)],
+                         ids=["f32", "bf16", "518x378"])
+def test_frame_attention_batch_is_per_frame_dense_attention(w):
+    """F frames in one call: frame f's tokens attend to frame f's tokens only.
+    bf16 device tensors go in one launch (one CTA per frame, tile pair and
+    head); its output equals the single-frame call's bit for bit (same split:
+    a frame's heads are short walks, never split) and the oracle's within the
+    tolerance.  fp32 and host tensors take one call per frame."""
+    cache = gca.Cache.for_workload(w, max_frames=8)
+    mirror = Mirror(w, [0])
+    F = 5 if w.Lq <= 64 else 3
+    rows = None if w.Lq <= 64 else _rows_sample(w.Lq, extra=4, seed=11)
+    q, k, v = (torch.stack([inputs.draw(w, 200 + f, x, "cuda")[0] for f in range(F)]) for x in "qkv")
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    n0 = cache.info().kernel_launches
+    cache.frame_attention_batch(0, q, k, v, out, lse)
+    launches = cache.info().kernel_launches - n0
+    assert launches == (1 if w.dtype == "bf16" else 2 * F)       # fp32: copy + attention per frame
+    for f in range(F):
+        o1 = torch.empty_like(q[f])
+        l1 = torch.empty(q.shape[1:3], dtype=torch.float32, device="cuda")
+        cache.frame_attention(0, q[f], k[f], v[f], o1, l1)
+        want, wlse = oracle_transient(mirror, 0, q[f].float().cpu().numpy(), k[f].float().cpu().numpy(),
+                                      v[f].float().cpu().numpy(), -1, rows=rows)
+        torch.cuda.synchronize()
+        assert torch.equal(out[f], o1) and torch.equal(lse[f], l1), f
+        got, gl = (out[f], lse[f]) if rows is None else (out[f][rows], lse[f][rows])
+        assert max_err(got, want) <= TOL[w.dtype], f
+        assert max_err(gl, wlse) <= LSE_TOL[w.dtype], f
+    # host tensors: staged one frame per launch, same values
+    out_h = torch.empty_like(q, device="cpu").pin_memory()
+    cache.frame_attention_batch(0, q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory(), out_h)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, out.cpu())
+    assert cache.info().frames == 0 and cache.status() == 0
+
+
 # ----------------------------------------------------------------------------
 # the larger workloads
 # ----------------------------------------------------------------------------

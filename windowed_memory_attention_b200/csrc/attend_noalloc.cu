@@ -225,14 +225,9 @@ extern "C" int gca_attend_pages_noalloc(const void* k_pool, const void* v_pool, 
     p.ws_o = ws_o;
     p.ws_lse = ws_lse;
     p.QT = QT;
-    const long long total = (long long)num_heads * nwalk;
-    long long w = std::max(1, sms / ((QT + 1) / 2));
-    w = std::min<long long>(w, (total + 3) / 4);
     // keep QT * (W + H - 1) partial tiles inside the scratch array
-    w = std::min<long long>(w, kNoallocMaxSlots / QT - num_heads + 1);
-    w = std::max<long long>(w, 1);
-    p.seg = (int)((total + w - 1) / w);
-    p.W = (int)((total + p.seg - 1) / p.seg);
+    gca::split_work(sms, (QT + 1) / 2, num_heads, nwalk, (long long)kNoallocMaxSlots / QT - num_heads + 1, &p.W,
+                    &p.seg);
     p.merge_cnt = counts;
     p.epoch = g_epoch.fetch_add(1) + 1;
     p.frame_page0 = INT_MAX;

@@ -311,7 +311,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // QK_t(j) (tile t, page j) writes S buffer (2j + t) % 3.  The buffer's previous
 // user is QK of index 2j + t - 3, whose PV is issued before QK_t(j), so each
 // tile's next S is computed while its softmax of the current page runs.
-template <int PAGE>
+template <int PAGE, bool BATCH>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               const __grid_constant__ CUtensorMap tmKf, const __grid_constant__ CUtensorMap tmVf,
@@ -355,6 +355,11 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int qp = blockIdx.x;
+    // batched frame attention: CTA row qp is tile pair qp % ppf of frame
+    // qp / ppf, which walks only that frame's own entries
+    const int bframe = BATCH ? qp / p.ppf : 0;
+    const int qpl = BATCH ? qp - bframe * p.ppf : qp;
+    const WalkEntry* const walk = p.walk + (BATCH ? (long long)bframe * p.nwalk : 0ll);
     const int w = blockIdx.y;
     const long long total = (long long)p.H * p.nwalk;
     const long long g0 = (long long)w * p.seg;
@@ -418,7 +423,7 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     ok = false;
                     break;
                 }
-                const int4 ent = __ldg(&p.walk[e]);
+                const int4 ent = __ldg(&walk[e]);
                 const int page = ent.x;
                 if (page < 0 || page >= p.num_pages) {
                     *abort_flag = 1;
@@ -532,9 +537,10 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         const int t = warp >> 2;
         const int quarter = warp & 3;
         const int rl = quarter * 32 + lane;
-        const int row = (qp * 2 + t) * kRows + rl;
-        const bool valid = row < p.R;
-        const int qframe = p.first_query_frame + (valid ? row / p.Lq : 0);
+        const int row_l = (qpl * 2 + t) * kRows + rl;
+        const int row = BATCH ? bframe * p.Lq + row_l : row_l;
+        const bool valid = BATCH ? row_l < p.Lq : row < p.R;
+        const int qframe = p.first_query_frame + (BATCH ? bframe : (valid ? row / p.Lq : 0));
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t t_o = tmem + lane_base + 3 * PAGE + t * 64;
         const float sl2 = p.scale_log2;
@@ -582,7 +588,7 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         int hd = 0;                                    // heads finished (o_done phases)
         int mg = 0;                                    // fused merges done (mrg_all / mrg_flag phases)
         load_q(h_start, 0);
-        int4 ent_next = __ldg(&p.walk[e_start]);
+        int4 ent_next = __ldg(&walk[e_start]);
         int h = h_start, e = e_start - 1;
         for (int j = 0; j < J; ++j) {
             if (++e == p.nwalk) {
@@ -600,7 +606,7 @@ attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 ++hs;
             }
             const int4 ent = ent_next;
-            if (j + 1 < J) ent_next = __ldg(&p.walk[e + 1 == p.nwalk ? 0 : e + 1]);
+            if (j + 1 < J) ent_next = __ldg(&walk[e + 1 == p.nwalk ? 0 : e + 1]);
             const int nvis = visible_prefix(p.rule, ent, qframe);
             const int b = (2 * j + t) % 3;
             const uint32_t t_s = tmem + lane_base + b * PAGE;
@@ -842,15 +848,15 @@ __global__ void bounded_wait_selftest(int* status, unsigned long long timeout_ns
     wait_bar(smem_u32(&bar), 0, ctl, true, timeout_ns);
 }
 
-template <int PAGE>
+template <int PAGE, bool BATCH>
 cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkf,
                         const CUtensorMap& tvf, const AttendParams& p, cudaStream_t s) {
     const int smem = Layout<PAGE>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(attend_kernel<PAGE>,
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel<PAGE, BATCH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((p.QT + 1) / 2, p.W);
-    attend_kernel<PAGE><<<grid, kThreads, smem, s>>>(tk, tv, tkf, tvf, p);
+    attend_kernel<PAGE, BATCH><<<grid, kThreads, smem, s>>>(tk, tv, tkf, tvf, p);
     return cudaGetLastError();
 }
 
@@ -858,8 +864,13 @@ cudaError_t launch_page(const CUtensorMap& tk, const CUtensorMap& tv, const CUte
 
 cudaError_t launch_attend_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkf,
                                 const CUtensorMap& tvf, const AttendParams& p, cudaStream_t s) {
-    if (p.P == 128) return launch_page<128>(tk, tv, tkf, tvf, p, s);
-    if (p.P == 64) return launch_page<64>(tk, tv, tkf, tvf, p, s);
+    if (p.ppf > 0) {
+        if (p.P == 128) return launch_page<128, true>(tk, tv, tkf, tvf, p, s);
+        if (p.P == 64) return launch_page<64, true>(tk, tv, tkf, tvf, p, s);
+        return cudaErrorInvalidValue;
+    }
+    if (p.P == 128) return launch_page<128, false>(tk, tv, tkf, tvf, p, s);
+    if (p.P == 64) return launch_page<64, false>(tk, tv, tkf, tvf, p, s);
     return cudaErrorInvalidValue;
 }
 

@@ -43,6 +43,7 @@ namespace {
 constexpr int kRing = 4;       // pinned staging slots for walk-list uploads
 constexpr int kQRing = 8;      // device staging slots for host query blocks
 constexpr int kORing = 2;      // device staging slots for host output blocks
+constexpr int kMaxBatch = 64;  // frames per launch of batched frame attention
 constexpr int kTileRows = 128;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -91,6 +92,7 @@ struct gca_cache {
     int up_n = 0;
     WalkEntry* d_walk_t = nullptr;   // walk list of the transient (non-keyframe) attention
     WalkEntry* d_walk_f = nullptr;   // the transient pages alone (frame attention)
+    WalkEntry* d_walk_b = nullptr;   // kMaxBatch frames' own pages (batched frame attention)
     unsigned long long tup_version = 0;
     int tup_n = 0;
     float* ws_o = nullptr;
@@ -149,6 +151,7 @@ void release(gca_cache* c) {
     cudaFree(c->d_walk);
     cudaFree(c->d_walk_t);
     cudaFree(c->d_walk_f);
+    cudaFree(c->d_walk_b);
     cudaFree(c->ws_o);
     cudaFree(c->ws_lse);
     cudaFree(c->merge_cnt);
@@ -310,10 +313,10 @@ bool encode_pool_map(EncodeTiledFn enc, CUtensorMap* tm, void* pool, const gca_c
 // tensor (D, H, token): a box of D x 1 x P is one head's tile of P tokens,
 // laid out in shared memory exactly like a pool page tile; boxes past the
 // last token read zeros.
-bool encode_frame_map(const gca_cache* c, CUtensorMap* tm, const void* base) {
+bool encode_frame_map(const gca_cache* c, CUtensorMap* tm, const void* base, int frames = 1) {
     if (!c->encode || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
     const cuuint64_t H = (cuuint64_t)c->cfg.num_heads;
-    cuuint64_t dims[3] = {(cuuint64_t)gca::kHeadDim, H, (cuuint64_t)c->Lq};
+    cuuint64_t dims[3] = {(cuuint64_t)gca::kHeadDim, H, (cuuint64_t)c->Lq * (cuuint64_t)frames};
     cuuint64_t strides[2] = {(cuuint64_t)gca::kHeadDim * 2, H * gca::kHeadDim * 2};
     cuuint32_t box[3] = {(cuuint32_t)gca::kHeadDim, 1, (cuuint32_t)c->P};
     cuuint32_t estr[3] = {1, 1, 1};
@@ -461,12 +464,7 @@ int run_attention(gca_cache* c, int layer, const void* q, int F, int first_query
     if (g.dtype == GCA_DTYPE_BF16) {
         // split: QT query tiles x W workers over the head-major page stream
         p.QT = ceil_div(R, kTileRows);
-        const long long total = (long long)g.num_heads * p.nwalk;
-        long long w = std::max(1, c->sms / ((p.QT + 1) / 2));   // CTAs = tile pairs x workers
-        w = std::min<long long>(w, (total + 3) / 4);
-        w = std::max<long long>(w, 1);
-        p.seg = ceil_div(total, w);
-        p.W = ceil_div(total, p.seg);
+        gca::split_work(c->sms, (p.QT + 1) / 2, g.num_heads, p.nwalk, LLONG_MAX, &p.W, &p.seg);
         p.merge_cnt = c->merge_cnt;
         p.epoch = ++c->epoch;
         p.frame_page0 = fk && fv ? c->num_regular : INT_MAX;
@@ -624,14 +622,23 @@ int gca_cache_create(const gca_config_t* cfg, int device, gca_cache_t** out) {
               cudaMalloc(&c->vpool, c->pool_bytes) == cudaSuccess;
     ok = ok && cudaMalloc(&c->d_walk, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
          cudaMalloc(&c->d_walk_t, sizeof(WalkEntry) * c->walk_cap) == cudaSuccess &&
-         cudaMalloc(&c->d_walk_f, sizeof(WalkEntry) * c->tpf) == cudaSuccess;
+         cudaMalloc(&c->d_walk_f, sizeof(WalkEntry) * c->tpf) == cudaSuccess &&
+         cudaMalloc(&c->d_walk_b, sizeof(WalkEntry) * c->tpf * kMaxBatch) == cudaSuccess;
     if (ok) {
-        // frame attention reads the transient pages only, as frame 0
-        std::vector<WalkEntry> wf(c->tpf);
+        // frame attention reads the transient pages only, as frame 0; the
+        // batched form gives frame f of a launch its own pages, whose tokens
+        // start at f * (S+M) of the caller's [F][S+M][H][D] tensors
+        std::vector<WalkEntry> wf(c->tpf), wb((size_t)c->tpf * kMaxBatch);
         for (int s = 0; s < c->tpf; ++s)
             wf[s] = make_int4(c->num_regular + s, std::min(c->P, c->Lq - s * c->P), s * c->P, 0);
+        for (int f = 0; f < kMaxBatch; ++f)
+            for (int s = 0; s < c->tpf; ++s)
+                wb[(size_t)f * c->tpf + s] = make_int4(c->num_regular + s, std::min(c->P, c->Lq - s * c->P),
+                                                       f * c->Lq + s * c->P, f);
         ok = cudaMemcpy(c->d_walk_f, wf.data(), sizeof(WalkEntry) * c->tpf, cudaMemcpyHostToDevice) ==
-             cudaSuccess;
+                 cudaSuccess &&
+             cudaMemcpy(c->d_walk_b, wb.data(), sizeof(WalkEntry) * wb.size(), cudaMemcpyHostToDevice) ==
+                 cudaSuccess;
     }
     for (int i = 0; ok && i < kRing; ++i) {
         ok = cudaHostAlloc((void**)&c->h_stage[i], sizeof(WalkEntry) * c->walk_cap, cudaHostAllocDefault) == cudaSuccess &&
@@ -953,6 +960,77 @@ int gca_frame_attention(gca_cache_t* c, int32_t layer, const void* q, const void
                            direct ? &fv : nullptr);
     if (direct && rc == GCA_OK && cudaEventRecord(c->kv_free, ex) != cudaSuccess) rc = GCA_ERR_CUDA;
     return end_call(c, st, ex, rc);
+}
+
+int gca_frame_attention_batch(gca_cache_t* c, int32_t layer, int32_t num_frames, const void* q, const void* k,
+                              const void* v, void* out, float* lse, void* stream) {
+    Range range("gca_frame_attention_batch");
+    if (!c || !q || !k || !v || !out || num_frames < 1) return GCA_ERR_INVALID_ARG;
+    if (c->host_only) return GCA_ERR_UNSUPPORTED;
+    const gca_config_t& g = c->cfg;
+    if (layer < 0 || layer >= g.num_layers) return GCA_ERR_INVALID_ARG;
+    if (!placed(q, 16) || !placed(k, 16) || !placed(v, 16) || !placed(out, 16) || !placed(lse, 4))
+        return GCA_ERR_INVALID_ARG;
+    if (int s = check_status(c)) return s;
+    const size_t fb = (size_t)c->Lq * g.num_heads * gca::kHeadDim * c->elem;
+    const size_t lb = (size_t)c->Lq * g.num_heads * sizeof(float);
+    auto at = [](const void* base, size_t off) { return static_cast<const char*>(base) + off; };
+    const bool batched = g.dtype == GCA_DTYPE_BF16 && g.rope == GCA_ROPE_NONE && !on_host(q) && !on_host(k) &&
+                         !on_host(v) && !on_host(out) && (!lse || !on_host(lse));
+    if (!batched) {
+        // host tensors (staged per frame), an fp32 cache or RoPE (K copied and
+        // rotated into the transient pages): one frame per launch
+        for (int f = 0; f < num_frames; ++f)
+            if (int rc = gca_frame_attention(c, layer, at(q, f * fb), at(k, f * fb), at(v, f * fb),
+                                             const_cast<char*>(at(out, f * fb)),
+                                             lse ? (float*)const_cast<char*>(at(lse, f * lb)) : nullptr, stream))
+                return rc;
+        return GCA_OK;
+    }
+    DeviceGuard guard(c->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int ppf = (ceil_div(c->Lq, kTileRows) + 1) / 2;    // tile pairs per frame
+    for (int f0 = 0; f0 < num_frames; f0 += kMaxBatch) {
+        const int n = std::min(kMaxBatch, num_frames - f0);
+        CUtensorMap fk{}, fv{};
+        if (!encode_frame_map(c, &fk, at(k, f0 * fb), n) || !encode_frame_map(c, &fv, at(v, f0 * fb), n))
+            return GCA_ERR_CUDA;
+        gca::AttendParams p{};
+        p.walk = c->d_walk_b;
+        p.nwalk = c->tpf;
+        p.q = at(q, f0 * fb);
+        p.out = const_cast<char*>(at(out, f0 * fb));
+        p.lse = lse ? (float*)const_cast<char*>(at(lse, f0 * lb)) : nullptr;
+        p.R = n * c->Lq;
+        p.H = g.num_heads;
+        p.Lq = c->Lq;
+        p.first_query_frame = 0;
+        p.rule = {g.num_anchor, g.window, c->keep, g.anchor_block ? 1 : 0};
+        p.scale = c->scale;
+        p.scale_log2 = c->scale * 1.4426950408889634f;
+        p.layer = layer;
+        p.num_pages = c->num_pages;
+        p.P = c->P;
+        p.status = c->d_status;
+        p.ws_o = c->ws_o;
+        p.ws_lse = c->ws_lse;
+        p.rope = c->rope();
+        // one CTA per (frame, tile pair, head): a frame's heads are a few pages
+        // each, so none is split and no partial or merge is needed
+        p.ppf = ppf;
+        p.QT = n * 2 * ppf;
+        p.W = g.num_heads;
+        p.seg = c->tpf;
+        p.merge_cnt = c->merge_cnt;
+        p.epoch = ++c->epoch;
+        p.frame_page0 = c->num_regular;
+        if (gca::launch_attend_sm100(c->tmK, c->tmV, fk, fv, p, st) != cudaSuccess) {
+            cudaGetLastError();
+            return GCA_ERR_CUDA;
+        }
+        c->launches += 1;
+    }
+    return GCA_OK;
 }
 
 int gca_attend_transient(gca_cache_t* c, int32_t layer, const void* q, const void* k, const void* v,

@@ -112,7 +112,32 @@ struct AttendParams {
     // frame tensor maps (token `first` of the walk entry onwards) instead of
     // the pools.  INT_MAX when unused.
     int frame_page0;
+    // batched frame attention (ppf > 0): R = F * Lq rows, F frames each with
+    // ppf tile pairs; frame f's tile pairs walk only its own nwalk entries at
+    // walk + f * nwalk, and its rows are frame first_query_frame + f
+    int ppf;
 };
+
+// Work split of the bf16 attention kernel: `pairs` query-tile pairs times W
+// workers, each worker a contiguous segment of `seg` entries of the
+// head-major (head, walk entry) stream.  One wave of CTAs (pairs * W <= SMs),
+// at least 4 entries per segment, W <= max_w.  A head whose walk is short
+// (kShortWalk pages or fewer) is not split when one CTA per (pair, head) fits
+// in a wave: splitting it costs more in pipeline fill, partial writes and the
+// merge than its few pages take (one 518x378 frame: 25 us unsplit, 37 us
+// split four ways).
+constexpr int kShortWalk = 12;
+inline void split_work(int sms, int pairs, int H, int nwalk, long long max_w, int* W, int* seg) {
+    const long long total = (long long)H * nwalk;
+    long long w = sms / pairs > 1 ? sms / pairs : 1;
+    w = w < (total + 3) / 4 ? w : (total + 3) / 4;
+    w = w < max_w ? w : max_w;
+    w = w > 1 ? w : 1;
+    long long s = (total + w - 1) / w;
+    if (s < nwalk && nwalk <= kShortWalk && (long long)pairs * H <= sms) s = nwalk;
+    *seg = (int)s;
+    *W = (int)((total + s - 1) / s);
+}
 
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);

@@ -29,6 +29,7 @@ EXPORTS = ("gca_cache_create", "gca_cache_destroy", "gca_append_frame", "gca_evi
            "gca_attend", "gca_reset", "gca_get_layout", "gca_token_slot", "gca_get_info",
            "gca_device_status", "gca_status_string", "gca_attend_pages_noalloc",
            "gca_selftest_bounded_wait", "gca_attend_transient", "gca_frame_attention",
+           "gca_frame_attention_batch",
            "gca_visible_prefix")
 
 
@@ -80,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "gca_attend": [vp, i32, vp, i32, vp, vp, vp],
             "gca_attend_transient": [vp, i32, vp, vp, vp, vp, vp, vp],
             "gca_frame_attention": [vp, i32, vp, vp, vp, vp, vp, vp],
+            "gca_frame_attention_batch": [vp, i32, i32, vp, vp, vp, vp, vp, vp],
             "gca_visible_prefix": [vp, ctypes.POINTER(gca_page_entry_t), i32, ctypes.POINTER(i32)],
             "gca_reset": [vp],
             "gca_get_layout": [vp, i32, ctypes.POINTER(gca_page_entry_t), i32, ctypes.POINTER(i32)],
@@ -177,6 +179,14 @@ def gca_frame_attention(cache, layer: int, q: torch.Tensor, k: torch.Tensor, v: 
                                                             _ptr(out), _ptr(lse), _stream(stream)))
 
 
+def gca_frame_attention_batch(cache, layer: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              out: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None) -> None:
+    """q, k, v, out: [F][S+M][H][D]; lse: [F][S+M][H]."""
+    _check("gca_frame_attention_batch",
+           lib().gca_frame_attention_batch(cache, layer, q.shape[0], _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                           _ptr(lse), _stream(stream)))
+
+
 def gca_reset(cache) -> None:
     _check("gca_reset", lib().gca_reset(cache))
 
@@ -269,6 +279,9 @@ class Cache:
 
     def frame_attention(self, layer, q, k, v, out, lse=None, stream=None):
         gca_frame_attention(self.handle, layer, q, k, v, out, lse, stream)
+
+    def frame_attention_batch(self, layer, q, k, v, out, lse=None, stream=None):
+        gca_frame_attention_batch(self.handle, layer, q, k, v, out, lse, stream)
 
     def reset(self):
         gca_reset(self.handle)
