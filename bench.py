@@ -62,6 +62,10 @@ def parse():
                     help="instead of the bench line: the CPU oracle's time per layer-step at the "
                          "report points (worked example and 518x378 at T=100/1000/10000, dense "
                          "limit at T=1000) on the host cores; no GPU work")
+    ap.add_argument("--frame-probe", type=int, default=0, metavar="FRAMES",
+                    help="instead of the bench line: intra-frame attention of the 518x378 workload, "
+                         "FRAMES frames per gca_frame_attention_batch call, 5 calls; a small command "
+                         "for profiler captures of the batched launch")
     ap.add_argument("--append-probe", type=int, default=0, metavar="FRAMES",
                     help="instead of the bench line: FRAMES appends of the 518x378 workload's 24 "
                          "layers into a small cache (window 4, about 1 GB of pools) with the append "
@@ -502,6 +506,23 @@ def run_append_probe(args):
                       "frac_hbm": b / (med / 1e3) / 1e9 / pk["hbm"]}), flush=True)
 
 
+def run_frame_probe(args):
+    """Batched intra-frame attention: 5 calls of FRAMES frames of one layer."""
+    dev = torch.device("cuda", 0)
+    w = inputs.METRIC_518x378.with_(L=1)
+    F = args.frame_probe
+    cache = gca.Cache.for_workload(w, max_frames=4)
+    q, k, v = (torch.stack([inputs.draw(w, f, x, dev)[0] for f in range(F)]) for x in "qkv")
+    out = torch.empty_like(q)
+    ms = _time_ms(lambda: cache.frame_attention_batch(0, q, k, v, out), reps=2, warm=3)
+    if cache.status() != 0:
+        raise RuntimeError("device status word raised")
+    fl = 4.0 * w.Lq * w.Lq * w.H * w.D * F
+    print(json.dumps({"frame_probe": w.name, "frames": F, "ms_per_call": ms, "ms_per_frame": ms / F,
+                      "tflops": fl / ms / 1e9}), flush=True)
+    cache.close()
+
+
 def run_oracle_report(args):
     """cpu_baseline of the report points: the oracle's attention core as it stands, on a bounded
     sample (64 query rows of one head) of each point's shape, scaled to all rows and heads.  The
@@ -690,6 +711,9 @@ def main():
         return
     if args.vo:
         run_vo_stream(torch.device("cuda", local_rank))
+        return
+    if args.frame_probe:
+        run_frame_probe(args)
         return
     if args.append_probe:
         run_append_probe(args)
