@@ -33,6 +33,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from windowed_memory_attention_b200 import gca, inputs  # noqa: E402
@@ -207,7 +208,7 @@ class OracleSample:
         t0 = time.perf_counter()
         kk, vv = ogca.gather_keys(last, fkv, n=w.n, k=w.k, S=w.S)
         t1 = time.perf_counter()
-        ogca.attention(q0[rows], kk, vv, w.softmax_scale)
+        self.last_out, _ = ogca.attention(q0[rows], kk, vv, w.softmax_scale)
         t2 = time.perf_counter()
         return t1 - t0, t2 - t1
 
@@ -447,6 +448,11 @@ def run_ours(args, rank, world, local_rank):
         g = sum(r[0] for r in runs) / len(runs)
         a = sum(r[1] for r in runs) / len(runs)
         step_s = g + a * w.Lq / len(rows)
+        # the same sample checks the timed step's output: layer 0 of frame T-1
+        got = out[0, 0].double().cpu().numpy()[rows]
+        line["parity"] = {"max_abs_err": float(np.abs(got - sample.last_out).max()), "tolerance": 2e-2,
+                          "rows": len(rows), "heads": w.H, "layer": 0, "frame": T_end - 1,
+                          "against": "CPU oracle (fp64) on the sampled rows"}
         from oracle import gca as ogca
         line["cpu_baseline"] = {
             "value": 1.0 / step_s, "unit": UNIT, "cores": ogca.core_threads(),
