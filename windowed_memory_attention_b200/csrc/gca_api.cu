@@ -989,6 +989,8 @@ int gca_frame_attention_batch(gca_cache_t* c, int32_t layer, int32_t num_frames,
     }
     DeviceGuard guard(c->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStream_t ex;
+    if (!begin_call(c, st, false, &ex)) return GCA_ERR_CUDA;   // device tensors: the caller's stream order
     const int ppf = (ceil_div(c->Lq, kTileRows) + 1) / 2;    // tile pairs per frame
     for (int f0 = 0; f0 < num_frames; f0 += kMaxBatch) {
         const int n = std::min(kMaxBatch, num_frames - f0);
@@ -1024,7 +1026,7 @@ int gca_frame_attention_batch(gca_cache_t* c, int32_t layer, int32_t num_frames,
         p.merge_cnt = c->merge_cnt;
         p.epoch = ++c->epoch;
         p.frame_page0 = c->num_regular;
-        if (gca::launch_attend_sm100(c->tmK, c->tmV, fk, fv, p, st) != cudaSuccess) {
+        if (gca::launch_attend_sm100(c->tmK, c->tmV, fk, fv, p, ex) != cudaSuccess) {
             cudaGetLastError();
             return GCA_ERR_CUDA;
         }
